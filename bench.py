@@ -1,0 +1,343 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 x FP4 MoE layer forward on B200.
+
+One step = moe_plan + moe_forward (permute -> linear1 + SwiGLU + requant ->
+linear2 x top-k weight -> combine) over one batch of the workload, inputs
+resident in HBM, L2 flushed (256 MB write) before every timed step.  Times
+are CUDA events on the launching stream.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mid]
+                  [--impl ours|reference]
+
+Multi-GPU: replicas (each rank runs its own batch of the workload with its
+own activations; no collective on the data path); the step time is the max
+over ranks and `value` counts the work of every rank ("scaling": "weak").
+`--impl reference` times the CPU oracle (the only reference this method has)
+on a bounded sample of the same workload, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer fwd TFLOPS & tokens/s on 1 B200; % of tensor/HBM roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="mid")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the bounded oracle sample")
+    return p.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, src="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws == 1:
+        return None, 0, 1, 0
+    import torch.distributed as dist
+    from datetime import timedelta
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    return dist, dist.get_rank(), ws, int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def _workload_desc(wl):
+    return (f"{wl.name}: T={wl.T} H={wl.H} I={wl.I} E={wl.E} top{wl.k} "
+            f"(W1 [{wl.E},{2 * wl.I},{wl.H}], W2 [{wl.E},{wl.H},{wl.I}] FP4 E2M1 + UE8M0/1x32; "
+            f"x FP8 E4M3 + UE8M0/1x32)")
+
+
+# ------------------------------------------------------------- CPU oracle
+def _oracle_sample(wl, inputs, seconds: float, rng_seed=0):
+    """Time the oracle on a bounded token sample; returns (TFLOPS, tokens, s, cores)."""
+    import numpy as np
+
+    import oracle
+    cores = oracle.max_threads()
+    rng = np.random.default_rng(rng_seed)
+    n = max(2, min(wl.T, cores))
+    toks = rng.choice(wl.T, n, replace=False).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.moe_forward(**inputs, tokens=toks)
+    dt = time.perf_counter() - t0
+    n2 = int(min(wl.T, max(n, n * seconds / max(dt, 1e-6))))
+    if n2 > n:
+        toks = rng.choice(wl.T, n2, replace=False).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.moe_forward(**inputs, tokens=toks)
+        dt = time.perf_counter() - t0
+        n = n2
+    flops = 6.0 * n * wl.k * wl.H * wl.I
+    return flops / dt / 1e12, n, dt, cores
+
+
+def run_reference(args, wl, rank):
+    """The reference arm: the CPU oracle, as it stands, on a bounded sample."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    import synth
+    inputs = synth.make_inputs(wl)
+    cores = oracle.max_threads()
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    # calibrate a per-step token sample
+    rng = np.random.default_rng(0)
+    n = max(2, min(wl.T, cores))
+    t0 = time.perf_counter()
+    oracle.moe_forward(**inputs, tokens=rng.choice(wl.T, n, replace=False).astype(np.int32))
+    dt = time.perf_counter() - t0
+    n = int(min(wl.T, max(2, n * per_step / max(dt, 1e-6))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        toks = rng.choice(wl.T, n, replace=False).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.moe_forward(**inputs, tokens=toks)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = statistics.mean(times)
+    flops = 6.0 * n * wl.k * wl.H * wl.I
+    value = flops / sec / 1e12
+    sample = f"{n} random tokens of {wl.T} per step (all their top-{wl.k} slots)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "tokens_per_s": n / sec, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+        "config": {"workload": _workload_desc(wl)},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ------------------------------------------------------------------ ours
+def run_ours(args, wl, dist, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import block_scaled_fp8_permute_b200 as moe
+    import synth
+    from tests.gpu_util import Layer
+
+    torch.cuda.set_device(local_rank)
+    dev = f"cuda:{local_rank}"
+    # each replica: shared weights, its own activations / routing
+    wl_r = wl if rank == 0 else synth.Workload(**{**wl.__dict__, "seed": wl.seed + rank})
+    x, x_sf, idx, tw = synth.make_activations(wl_r)
+    w1, w1_sf, w2, w2_sf = synth.make_weights(wl)
+    inputs = dict(x=x, x_sf=x_sf, topk_idx=idx, topk_w=tw, w1=w1, w1_sf=w1_sf, w2=w2, w2_sf=w2_sf)
+    lay = Layer(inputs, device=dev)
+    shp, d = lay.shape, lay.dev
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        moe.moe_plan(shp, d["topk_idx"], lay.ws)
+        moe.moe_forward(shp, d["x"], d["x_sf"], d["topk_idx"], d["topk_w"], *lay.wt, lay.y,
+                        lay.ws)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(lay.ws) == 0, "device status after warm-up"
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(K)]
+    for row in ev:
+        for e in row:
+            e.record(stream)  # materialise the handles
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(K):
+            flush.zero_()
+            moe.moe_set_timing_events(ev[i][1:6])
+            ev[i][0].record(stream)
+            step()
+            ev[i][6].record(stream)
+        moe.moe_set_timing_events(None)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = [ev[i][0].elapsed_time(ev[i][6]) for i in range(K)]
+    kern = {name: statistics.mean(ev[i][a].elapsed_time(ev[i][b]) for i in range(K))
+            for name, a, b in (("plan", 0, 1), ("permute", 1, 2), ("linear1", 2, 3),
+                               ("linear2", 3, 4), ("combine", 4, 5))}
+    ms = statistics.mean(step_ms)
+    status = moe.moe_get_device_status(lay.ws)
+    assert status == 0, f"device status {status}"
+
+    # e2e: the host-buffer entry point, host<->device copies inside the timed region
+    ws_h = moe.alloc_workspace(shp, dev, host_variant=True)
+    pin = {k: torch.from_numpy(np.ascontiguousarray(inputs[k])).pin_memory()
+           for k in ("x", "x_sf", "topk_idx", "topk_w")}
+    y_host = torch.empty((wl.T, wl.H), dtype=torch.int16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = y_host.numel() * y_host.element_size()
+    e2e_ms = []
+    for i in range(max(args.warmup, 3) + K):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        moe.moe_forward_host(shp, pin["x"], pin["x_sf"], pin["topk_idx"], pin["topk_w"], *lay.wt,
+                             y_host, ws_h)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= max(args.warmup, 3):
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e = statistics.mean(e2e_ms)
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    ms = max_over_ranks(ms)
+    e2e = max_over_ranks(e2e)
+    g1 = max_over_ranks(kern["linear1"])
+    if rank != 0:
+        return
+    flops = wl.flops * world
+    value = flops / (ms * 1e-3) / 1e12
+    pk = _peaks()
+    tensor_peak = 2.0 * pk["bf16"]  # FP8-rate MMA = 2 x the measured bf16 rate
+    g1_flops = 4.0 * wl.R * wl.H * wl.I
+    g1_tflops = g1_flops / (g1 * 1e-3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline:
+        cv, n, sec, cores = _oracle_sample(wl, inputs, args.cpu_seconds)
+        cpu = {"value": cv, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+               "sample": f"{n} random tokens of {wl.T} (all top-{wl.k} slots), {sec:.1f} s"}
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "tokens_per_s": wl.T * world / (ms * 1e-3),
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3 x fp4_e2m1, fp32 accumulate, bf16 out", "data": "synthetic",
+        "config": {"workload": _workload_desc(wl), "tokens_per_gpu": wl.T,
+                   "l2": "flushed (256 MB write) before every timed step",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "linear1 (moe_gemm_kernel<1>)",
+                     "achieved": g1_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
+                     "frac": g1_tflops / tensor_peak, "traffic": None,
+                     "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"},
+        "kernels_ms": kern,
+        "step_roofline_frac": (wl.flops / (ms * 1e-3) / 1e12) / tensor_peak,
+        "e2e": {"value": flops / (e2e * 1e-3) / 1e12, "unit": "TFLOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+        "gpu_launches": 7 * K,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = _args()
+    import synth
+    wl = synth.workload(args.workload)
+    if args.impl == "reference":
+        # the CPU oracle runs on rank 0 only; other ranks leave at once
+        run_reference(args, wl, int(os.environ.get("RANK", "0")))
+        return
+    dist, rank, world, local_rank = _dist()
+    try:
+        run_ours(args, wl, dist, rank, world, local_rank)
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

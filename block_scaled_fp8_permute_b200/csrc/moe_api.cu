@@ -1,0 +1,412 @@
+// moe_api.cu -- the extern "C" entry points of libmoe (declared in
+// include/moe.h): argument validation, workspace carving, tensor-map
+// encoding and the launch sequence of one MoE layer forward.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                        const GemmArgs& args, int grid, bool pdl, cudaStream_t stream);
+cudaError_t launch_requant_debug(const float* a, int rows, int cols, uint8_t* codes,
+                                 uint8_t* sbytes, cudaStream_t stream);
+cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int* chunk, int* counts,
+                        int* offs, int* poffs, int* tile_expert, int* row_of, int* src_of,
+                        int* hdr, cudaStream_t stream);
+cudaError_t launch_permute(const uint8_t* x, const int32_t* x_sf, const int* src_of,
+                           const int* hdr, int H, int topk, uint8_t* xp, uint8_t* xp_sf, int grid,
+                           bool pdl, cudaStream_t stream);
+cudaError_t launch_combine(const float* yp, const int* row_of, int T, int H, int topk, uint16_t* y,
+                           int grid, bool pdl, cudaStream_t stream);
+cudaError_t launch_transform(const uint8_t* w, const uint8_t* w_sf, int E, int N, int K,
+                             int interleave, uint8_t* wt, uint8_t* wt_sf, cudaStream_t stream);
+
+namespace {
+
+std::atomic<int> g_num_sms_cap{0};
+std::atomic<int> g_pdl{1};
+std::mutex g_ev_mu;
+cudaEvent_t g_events[5];
+bool g_events_on = false;
+
+void record_event(int i, cudaStream_t s) {
+  std::lock_guard<std::mutex> lk(g_ev_mu);
+  if (g_events_on) cudaEventRecord(g_events[i], s);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  int cap = g_num_sms_cap.load();
+  return (cap > 0 && cap < n) ? cap : n;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status check_shape(const moe_shape* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->E <= 0 || s->topk <= 0)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s->H % 128 || s->I % 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (s->E > kMaxE || s->topk > kMaxTopk || s->topk > s->E) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)s->T * s->topk > (1LL << 24)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)s->H * s->I > (1LL << 31) || s->H > 65536 || s->I > 65536)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+// activations [rows, K] uint8 E4M3: box 128 x 128, 128-byte swizzle
+bool encode_act(CUtensorMap* m, const void* base, int rows, int K) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K};
+  cuuint32_t box[2] = {128, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// transformed weights [E*KB][n_rows][128 E2M1 = 64 bytes]: box 128 x 256 x 1;
+// the TMA unpacks every 16 codes (8 bytes) into a 16-byte shared-memory slot.
+bool encode_wgt(CUtensorMap* m, const void* base, int E, int KB, int n_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)n_rows, (cuuint64_t)E * KB};
+  cuuint64_t strides[2] = {64, (cuuint64_t)n_rows * 64};
+  cuuint32_t box[3] = {128, 256, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Ws {
+  WsLayout L;
+  uint8_t* base;
+  int* hdr() const { return reinterpret_cast<int*>(base + L.hdr); }
+  int* counts() const { return reinterpret_cast<int*>(base + L.counts); }
+  int* offs() const { return reinterpret_cast<int*>(base + L.offs); }
+  int* poffs() const { return reinterpret_cast<int*>(base + L.poffs); }
+  int* chunk() const { return reinterpret_cast<int*>(base + L.chunk); }
+  int* row_of() const { return reinterpret_cast<int*>(base + L.row_of); }
+  int* src_of() const { return reinterpret_cast<int*>(base + L.src_of); }
+  int* tile_expert() const { return reinterpret_cast<int*>(base + L.tile_expert); }
+  uint8_t* xp() const { return base + L.xp; }
+  uint8_t* xp_sf() const { return base + L.xp_sf; }
+  uint8_t* a2() const { return base + L.a2; }
+  uint8_t* a2_sf() const { return base + L.a2_sf; }
+  float* yp() const { return reinterpret_cast<float*>(base + L.yp); }
+};
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// staging area of moe_forward_host, after the regular workspace
+struct HostStage {
+  size_t x, x_sf, idx, w, y, total;
+};
+HostStage host_stage(const moe_shape& s, size_t base) {
+  HostStage h{};
+  size_t off = base;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  h.x = take((size_t)s.T * s.H);
+  h.x_sf = take((size_t)s.T * (s.H / 128) * 4);
+  h.idx = take((size_t)s.T * s.topk * 4);
+  h.w = take((size_t)s.T * s.topk * 4);
+  h.y = take((size_t)s.T * s.H * 2);
+  h.total = off;
+  return h;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_BAD_EXPERT_ID: return "MOE_ERR_BAD_EXPERT_ID";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int moe_block_m(void) { return kBlockM; }
+
+void moe_set_num_sms(int num_sms) { g_num_sms_cap.store(num_sms > 0 ? num_sms : 0); }
+
+void moe_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
+
+void moe_set_timing_events(void* const* events, int n) {
+  std::lock_guard<std::mutex> lk(g_ev_mu);
+  g_events_on = (events != nullptr && n >= 5);
+  if (g_events_on)
+    for (int i = 0; i < 5; ++i) g_events[i] = static_cast<cudaEvent_t>(events[i]);
+}
+
+size_t moe_transformed_bytes(const moe_shape* shape, int which, size_t* sf_bytes) {
+  if (check_shape(shape) != MOE_OK || (which != 1 && which != 2)) {
+    if (sf_bytes) *sf_bytes = 0;
+    return 0;
+  }
+  const size_t E = shape->E, H = shape->H, I = shape->I;
+  const size_t elems = (which == 1) ? E * 2 * I * H : E * H * I;
+  if (sf_bytes) *sf_bytes = elems / 32;
+  return elems / 2;
+}
+
+moe_status moe_transform_weights(const moe_shape* shape, const uint8_t* w1, const uint8_t* w1_sf,
+                                 const uint8_t* w2, const uint8_t* w2_sf, void* w1_t,
+                                 void* w1_sf_t, void* w2_t, void* w2_sf_t, moe_stream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  const void* ptrs[] = {w1, w1_sf, w2, w2_sf, w1_t, w1_sf_t, w2_t, w2_sf_t};
+  for (const void* p : ptrs)
+    if (!p || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {(const void*)w1_t, (const void*)w1_sf_t, (const void*)w2_t,
+                        (const void*)w2_sf_t})
+    if (!aligned(p, 256)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_transform(w1, w1_sf, shape->E, 2 * shape->I, shape->H, 1,
+                                   static_cast<uint8_t*>(w1_t), static_cast<uint8_t*>(w1_sf_t), s);
+  if (e == cudaSuccess)
+    e = launch_transform(w2, w2_sf, shape->E, shape->H, shape->I, 0, static_cast<uint8_t*>(w2_t),
+                         static_cast<uint8_t*>(w2_sf_t), s);
+  return cuda_status(e);
+}
+
+size_t moe_workspace_bytes(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return ws_layout(*shape).total;
+}
+
+int moe_plan_max_rows(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return ws_layout(*shape).P_max;
+}
+
+moe_status moe_plan(const moe_shape* shape, const int32_t* topk_idx, void* workspace,
+                    size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  if (shape->T > 0 && (!topk_idx || !aligned(topk_idx, 4))) return MOE_ERR_INVALID_ARG;
+  Ws ws{ws_layout(*shape), static_cast<uint8_t*>(workspace)};
+  if (ws_bytes < ws.L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(ws.hdr(), 0, kHdrWords * 4, s);
+  if (e == cudaSuccess)
+    e = launch_plan(topk_idx, ws.L.R, shape->E, ws.L.NCH, ws.chunk(), ws.counts(), ws.offs(),
+                    ws.poffs(), ws.tile_expert(), ws.row_of(), ws.src_of(), ws.hdr(), s);
+  return cuda_status(e);
+}
+
+moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* x_sf,
+                       const int32_t* topk_idx, const float* topk_w, const void* w1_t,
+                       const void* w1_sf_t, const void* w2_t, const void* w2_sf_t, uint16_t* y,
+                       void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  const moe_shape sh = *shape;
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  Ws ws{ws_layout(sh), static_cast<uint8_t*>(workspace)};
+  if (ws_bytes < ws.L.total) return MOE_ERR_WORKSPACE;
+  if (sh.T == 0) return MOE_OK;
+  const void* p16[] = {x, x_sf, topk_w, y};
+  for (const void* p : p16)
+    if (!p || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const void* p256[] = {w1_t, w1_sf_t, w2_t, w2_sf_t};
+  for (const void* p : p256)
+    if (!p || !aligned(p, 256)) return MOE_ERR_INVALID_ARG;
+  if (!topk_idx || !aligned(topk_idx, 4)) return MOE_ERR_INVALID_ARG;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = device_sms();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  const bool pdl = g_pdl.load() != 0;
+  const int KB1 = sh.H / 128, KB2 = sh.I / 128;
+  const int NT1 = (2 * sh.I + kBlockN - 1) / kBlockN, NT2 = (sh.H + kBlockN - 1) / kBlockN;
+
+  CUtensorMap tmX, tmW1, tmA2, tmW2;
+  if (!encode_act(&tmX, ws.xp(), ws.L.P_max, sh.H) ||
+      !encode_wgt(&tmW1, w1_t, sh.E, KB1, 2 * sh.I) ||
+      !encode_act(&tmA2, ws.a2(), ws.L.P_max, sh.I) ||
+      !encode_wgt(&tmW2, w2_t, sh.E, KB2, sh.H))
+    return MOE_ERR_CUDA;
+
+  // dispatch: permute rows into expert-contiguous order
+  record_event(0, s);
+  int pgrid = (ws.L.P_max + 7) / 8;
+  if (pgrid > sms * 16) pgrid = sms * 16;
+  if (pgrid < 1) pgrid = 1;
+  cudaError_t e = launch_permute(x, x_sf, ws.src_of(), ws.hdr(), sh.H, sh.topk, ws.xp(),
+                                 ws.xp_sf(), pgrid, false, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  record_event(1, s);
+
+  GemmArgs g1{};
+  g1.sfa = ws.xp_sf();
+  g1.sfb = static_cast<const uint8_t*>(w1_sf_t);
+  g1.hdr = ws.hdr();
+  g1.tile_expert = ws.tile_expert();
+  g1.src_of = ws.src_of();
+  g1.KB = KB1;
+  g1.n_rows = 2 * sh.I;
+  g1.NT = NT1;
+  g1.a2 = ws.a2();
+  g1.a2_sf = ws.a2_sf();
+  g1.I = sh.I;
+  g1.H = sh.H;
+  long long tiles1 = (long long)ws.L.MT_max * NT1;
+  int grid1 = (int)(tiles1 < sms ? tiles1 : sms);
+  if (grid1 < 1) grid1 = 1;
+  e = launch_gemm(1, tmX, tmW1, g1, grid1, pdl, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  record_event(2, s);
+
+  GemmArgs g2 = g1;
+  g2.sfa = ws.a2_sf();
+  g2.sfb = static_cast<const uint8_t*>(w2_sf_t);
+  g2.KB = KB2;
+  g2.n_rows = sh.H;
+  g2.NT = NT2;
+  g2.yp = ws.yp();
+  g2.topk_w = topk_w;
+  long long tiles2 = (long long)ws.L.MT_max * NT2;
+  int grid2 = (int)(tiles2 < sms ? tiles2 : sms);
+  if (grid2 < 1) grid2 = 1;
+  e = launch_gemm(2, tmA2, tmW2, g2, grid2, pdl, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  record_event(3, s);
+
+  int cgrid = sh.T < 65535 ? sh.T : 65535;
+  e = launch_combine(ws.yp(), ws.row_of(), sh.T, sh.H, sh.topk, y, cgrid, pdl, s);
+  record_event(4, s);
+  return cuda_status(e);
+}
+
+size_t moe_workspace_bytes_host(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  WsLayout L = ws_layout(*shape);
+  return host_stage(*shape, L.total).total;
+}
+
+moe_status moe_forward_host(const moe_shape* shape, const uint8_t* x_host,
+                            const int32_t* x_sf_host, const int32_t* topk_idx_host,
+                            const float* topk_w_host, const void* w1_t, const void* w1_sf_t,
+                            const void* w2_t, const void* w2_sf_t, uint16_t* y_host,
+                            void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  const moe_shape sh = *shape;
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  WsLayout L = ws_layout(sh);
+  HostStage hs = host_stage(sh, L.total);
+  if (ws_bytes < hs.total) return MOE_ERR_WORKSPACE;
+  if (sh.T == 0) return MOE_OK;
+  if (!x_host || !x_sf_host || !topk_idx_host || !topk_w_host || !y_host)
+    return MOE_ERR_INVALID_ARG;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t nx = (size_t)sh.T * sh.H, nsf = (size_t)sh.T * (sh.H / 128) * 4,
+               nk = (size_t)sh.T * sh.topk * 4, ny = (size_t)sh.T * sh.H * 2;
+  cudaError_t e = cudaMemcpyAsync(base + hs.x, x_host, nx, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(base + hs.x_sf, x_sf_host, nsf, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(base + hs.idx, topk_idx_host, nk, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(base + hs.w, topk_w_host, nk, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const int32_t* idx_d = reinterpret_cast<const int32_t*>(base + hs.idx);
+  st = moe_plan(shape, idx_d, workspace, L.total, stream);
+  if (st != MOE_OK) return st;
+  st = moe_forward(shape, base + hs.x, reinterpret_cast<const int32_t*>(base + hs.x_sf), idx_d,
+                   reinterpret_cast<const float*>(base + hs.w), w1_t, w1_sf_t, w2_t, w2_sf_t,
+                   reinterpret_cast<uint16_t*>(base + hs.y), workspace, L.total, stream);
+  if (st != MOE_OK) return st;
+  e = cudaMemcpyAsync(y_host, base + hs.y, ny, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+moe_status moe_get_device_status(const void* workspace, moe_stream_t stream) {
+  if (!workspace) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  int hdr[kHdrWords];
+  if (cudaMemcpy(hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return static_cast<moe_status>(hdr[kHdrStatus]);
+}
+
+moe_status moe_plan_export(const moe_shape* shape, const void* workspace, int32_t* counts,
+                           int32_t* offs, int32_t* padded_offs, int32_t* row_of, int32_t* src_of,
+                           int32_t* P_out, moe_stream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!workspace || !counts || !offs || !padded_offs || !row_of || !P_out)
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  Ws ws{ws_layout(*shape), static_cast<uint8_t*>(const_cast<void*>(workspace))};
+  const int E = shape->E;
+  int hdr[kHdrWords];
+  cudaError_t e = cudaMemcpy(hdr, ws.hdr(), sizeof(hdr), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(counts, ws.counts(), E * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(offs, ws.offs(), (E + 1) * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(padded_offs, ws.poffs(), (E + 1) * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && ws.L.R > 0)
+    e = cudaMemcpy(row_of, ws.row_of(), (size_t)ws.L.R * 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  *P_out = hdr[kHdrP];
+  if (src_of && hdr[kHdrP] > 0) {
+    if (hdr[kHdrP] > ws.L.P_max) return MOE_ERR_CUDA;
+    if (cudaMemcpy(src_of, ws.src_of(), (size_t)hdr[kHdrP] * 4, cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_debug_requant(const float* a, int rows, int cols, uint8_t* codes, uint8_t* sbytes,
+                             moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!a || !codes || !sbytes || !aligned(a, 16) || !aligned(codes, 16))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_requant_debug(a, rows, cols, codes, sbytes,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

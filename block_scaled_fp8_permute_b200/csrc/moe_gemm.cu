@@ -1,0 +1,374 @@
+// moe_gemm.cu -- persistent grouped GEMM on 5th-generation tensor cores for
+// the two linear layers of the MoE layer.
+//
+//   linear1: G = Xp_e . W1_e^T  (FP8 E4M3 activations x FP4 E2M1 weights,
+//            UE8M0 scale per 1x32 block on both sides, FP32 accumulation) with
+//            the SwiGLU + E4M3 requantisation epilogue fused in;
+//   linear2: O = A2_e . W2_e^T with the top-k weight applied in the epilogue,
+//            FP32 partial rows written in expert-contiguous row order.
+// ("DeepSeek DeepGEMM 2026年4月重磅更新：Mega MoE融合算子、FP4精度与极致性能优化",
+//  section 3.2 (fusing linear1 / SwiGLU / linear2), section 4.2 (UE8M0 scale
+//  factors, FP32 accumulation), section 11.3 (TMA multi-stage loads).)
+//
+// One CTA per SM, 320 threads:
+//   warp 0     TMA producer: A tile 128x128 (E4M3), B tile 256x128 (E2M1,
+//              unpacked by the TMA to one byte per element as the block-scaled
+//              MMA requires), and the two 512/1024-byte scale chunks, into a
+//              4-stage shared-memory ring.
+//   warp 1     TMEM allocator and MMA issuer: copies the stage's scales into
+//              TMEM (tcgen05.cp) and issues 4 x tcgen05.mma kind::mxf8f6f4
+//              (M=128, N=256, K=32) per stage into one FP32 TMEM accumulator.
+//   warps 2-9  epilogue: drain the accumulator from TMEM (two warps per
+//              32-lane subpartition, one column half each), release it to
+//              the MMA warp, then compute and store.
+// Tiles: (m-tile of 128 padded rows, n-tile of 256 weight rows); each m-tile
+// belongs to one expert (rows are padded per expert to 128).
+#include <cuda_fp8.h>
+
+#include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+constexpr int kStages = 4;
+constexpr int kSmemA = kBlockM * kBlockK;  // 16384 bytes
+constexpr int kSmemB = kBlockN * kBlockK;  // 32768 bytes (one byte per E2M1 element in smem)
+constexpr int kTxB = kBlockN * kBlockK / 2;  // bytes the TMA moves for B (packed)
+constexpr int kSmemSFA = kSfChunk;
+constexpr int kSmemSFB = 2 * kSfChunk;
+constexpr int kNumEpiWarps = 8;
+constexpr int kGemmThreads = 64 + 32 * kNumEpiWarps;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCol = 0;    // FP32 accumulator, 256 columns
+constexpr uint32_t kSfCol = 256;   // scale buffers: buf b -> SFA at +16b (4 cols), SFB at +16b+4 (8)
+constexpr size_t kGemmSmemBytes =
+    1024 + (size_t)kStages * (kSmemA + kSmemB + kSmemSFA + kSmemSFB) + 256;
+
+// ------------------------------------------------------------- requantiser
+// Smallest e with 448 * 2^e >= amax, from the bits of amax (448 = 1.75 * 2^8):
+// amax = m * 2^x with m in [1,2) needs e = x - 8 when m <= 1.75, else x - 7.
+// amax == 0 gives 0; results are clamped to [-127, 127].
+__device__ __forceinline__ int e4m3_block_exponent(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  const int biased = (int)((bits >> 23) & 0xFF);
+  if (amax == 0.0f) return 0;
+  if (biased == 0) return -127;
+  const int x = biased - 127;
+  int e = ((bits & 0x7FFFFFu) > 0x600000u) ? x - 7 : x - 8;
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// Requantise 32 floats: E4M3 codes (little-endian packed, 4 per word) and
+// the UE8M0 byte of the block.
+__device__ __forceinline__ void requant32(const float (&a)[32], uint32_t (&packed)[8],
+                                          uint32_t& sbyte) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(a[i]));
+  const int e = e4m3_block_exponent(amax);
+  const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const __nv_fp8x2_storage_t lo =
+        __nv_cvt_float2_to_fp8x2(make_float2(a[4 * i] * inv, a[4 * i + 1] * inv), __NV_SATFINITE,
+                                 __NV_E4M3);
+    const __nv_fp8x2_storage_t hi =
+        __nv_cvt_float2_to_fp8x2(make_float2(a[4 * i + 2] * inv, a[4 * i + 3] * inv),
+                                 __NV_SATFINITE, __NV_E4M3);
+    packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+  }
+  sbyte = (uint32_t)(e + 127);
+}
+
+__global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int cols,
+                                     uint8_t* __restrict__ codes, uint8_t* __restrict__ sbytes) {
+  const int nblk = cols / 32;
+  for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < (long long)rows * nblk;
+       b += (long long)gridDim.x * blockDim.x) {
+    float v[32];
+    const float* src = a + b * 32;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = src[i];
+    uint32_t packed[8], sb;
+    requant32(v, packed, sb);
+    uint4* dst = reinterpret_cast<uint4*>(codes + b * 32);
+    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    sbytes[b] = (uint8_t)sb;
+  }
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// -------------------------------------------------------------------- kernel
+template <int kEpi>  // 1: SwiGLU + requant (linear1), 2: x topk_w, FP32 rows (linear2)
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+  using namespace ptx;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<size_t>(smem_raw), 1024));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + kStages * kSmemA;
+  uint8_t* sSFA = sB + kStages * kSmemB;
+  uint8_t* sSFB = sSFA + kStages * kSmemSFA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + kStages * kSmemSFB);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kNumEpiWarps);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  pdl_wait();  // inputs come from the previous kernel of the forward
+  const int NT = args.NT, KB = args.KB, n_rows = args.n_rows;
+  const int num_tiles = args.hdr[kHdrMTiles] * NT;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      uint32_t issued_mask = 0, last_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mt = tile / NT, nt = tile - (tile / NT) * NT;
+        const int e = args.tile_expert[mt];
+        const int n0 = nt * kBlockN;
+        const uint32_t sfb_bytes = (n_rows - n0 > 128) ? 2 * kSfChunk : kSfChunk;
+        const uint32_t tx = kSmemA + kTxB + kSfChunk + sfb_bytes;
+        const uint8_t* sfa_src = args.sfa + (size_t)mt * KB * kSfChunk;
+        const uint8_t* sfb_src = args.sfb + ((size_t)e * KB * (n_rows / 128) + n0 / 128) * kSfChunk;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
+            set_status(args.hdr, MOE_ERR_TIMEOUT);
+            args.hdr[kHdrTimeoutSite] = 10 + kEpi;
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], tx);
+          tma_load_2d(sA + s * kSmemA, &tmA, &full[s], kb * kBlockK, mt * kBlockM);
+          tma_load_3d(sB + s * kSmemB, &tmB, &full[s], 0, n0, e * KB + kb);
+          bulk_load(sSFA + s * kSmemSFA, sfa_src + (size_t)kb * kSfChunk, kSfChunk, &full[s]);
+          bulk_load(sSFB + s * kSmemSFB, sfb_src + (size_t)kb * (n_rows / 128) * kSfChunk,
+                    sfb_bytes, &full[s]);
+          issued_mask |= 1u << s;
+          last_phase = (last_phase & ~(1u << s)) | (ph << s);
+        }
+      }
+      if (!ok) {
+        // let copies already in flight land before the CTA's memory goes away
+        for (int s = 0; s < kStages; ++s)
+          if (issued_mask & (1u << s)) (void)mbar_wait(&full[s], (last_phase >> s) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      uint32_t it = 0;
+      int ti = 0;
+      bool issued_any = false, ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++ti) {
+        const int nt = tile % NT;
+        const int n_tile = min(kBlockN, n_rows - nt * kBlockN);
+        const uint32_t idesc0 = idesc_mxf8f6f4(/*A E4M3*/ 0, /*B E2M1*/ 5, kBlockM, n_tile);
+        if (!mbar_wait(acc_empty, (ti & 1) ^ 1) || *abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!mbar_wait(&full[s], ph) || *abort_flag) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sfa_t = tmem + kSfCol + 16u * (it & 1u);
+          const uint32_t sfb_t = sfa_t + 4u;
+          tc_cp_32x128b_warpx4(sfa_t, sdesc_sf(smem_u32(sSFA + s * kSmemSFA)));
+          tc_cp_32x128b_warpx4(sfb_t, sdesc_sf(smem_u32(sSFB + s * kSmemSFB)));
+          if (n_tile > 128)
+            tc_cp_32x128b_warpx4(sfb_t + 4u, sdesc_sf(smem_u32(sSFB + s * kSmemSFB + kSfChunk)));
+          const uint64_t adesc = sdesc_sw128(smem_u32(sA + s * kSmemA));
+          const uint64_t bdesc = sdesc_sw128(smem_u32(sB + s * kSmemB));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t id = idesc_with_sf_id(idesc0, kk, kk);
+            mma_mxf8f6f4(tmem + kAccCol, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id,
+                         (kb | kk) != 0 ? 1u : 0u, sfa_t | ((uint32_t)kk << 30),
+                         sfb_t | ((uint32_t)kk << 30));
+          }
+          issued_any = true;
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+      }
+      if (!ok) {
+        set_status(args.hdr, MOE_ERR_TIMEOUT);
+        args.hdr[kHdrTimeoutSite] = 20 + kEpi;
+        *abort_flag = 1;
+        if (issued_any) {  // wait for the MMAs in flight before TMEM is released
+          tc_commit(drain);
+          (void)mbar_wait(drain, 0);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;      // 0..7
+    const int q = warp & 3;       // TMEM lane subpartition this warp can read
+    const int h = ew >> 2;        // column half
+    const int r = q * 32 + lane;  // row within the tile
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + kAccCol;
+    int ti = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++ti) {
+      const int mt = tile / NT, nt = tile - (tile / NT) * NT;
+      // warp-uniform decision: every lane leaves or every lane continues
+      const bool ready = __all_sync(0xffffffffu, mbar_wait(acc_full, ti & 1) && !*abort_flag);
+      if (!ready) {
+        if (lane == 0) {
+          set_status(args.hdr, MOE_ERR_TIMEOUT);
+          args.hdr[kHdrTimeoutSite] = 30 + kEpi;
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      uint32_t v[4][32];
+      if (kEpi == 1) {
+        // gate columns [64h, 64h+64), up columns [128+64h, 128+64h+64)
+        tmem_ld_32x32b_x32(trow + 64 * h, v[0]);
+        tmem_ld_32x32b_x32(trow + 64 * h + 32, v[1]);
+        tmem_ld_32x32b_x32(trow + 128 + 64 * h, v[2]);
+        tmem_ld_32x32b_x32(trow + 128 + 64 * h + 32, v[3]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(trow + 128 * h + 32 * c, v[c]);
+      }
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+
+      const int row = mt * kBlockM + r;
+      const int src = args.src_of[row];
+      if (src < 0) continue;  // padding row (the loop head reconverges the warp)
+      if (kEpi == 1) {
+        uint32_t sbytes = 0;
+        uint8_t* dst = args.a2 + (size_t)row * args.I + nt * 128 + 64 * h;
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          float a[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float g = __uint_as_float(v[b][i]);
+            const float u = __uint_as_float(v[2 + b][i]);
+            a[i] = g / (1.0f + __expf(-g)) * u;
+          }
+          uint32_t packed[8], sb;
+          requant32(a, packed, sb);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * b);
+          d4[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          d4[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          sbytes |= sb << (8 * b);
+        }
+        uint8_t* sfdst = args.a2_sf + ((size_t)mt * (args.I / 128) + nt) * kSfChunk +
+                         (r & 31) * 16 + (r >> 5) * 4 + 2 * h;
+        *reinterpret_cast<uint16_t*>(sfdst) = (uint16_t)sbytes;
+      } else {
+        const int col0 = nt * kBlockN + 128 * h;
+        if (col0 >= n_rows) continue;  // half tile at the end of N
+        const float w = args.topk_w[src];
+        float4* dst = reinterpret_cast<float4*>(args.yp + (size_t)row * args.H + col0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[c * 8 + j] = make_float4(w * __uint_as_float(v[c][4 * j]),
+                                         w * __uint_as_float(v[c][4 * j + 1]),
+                                         w * __uint_as_float(v[c][4 * j + 2]),
+                                         w * __uint_as_float(v[c][4 * j + 3]));
+      }
+    }
+  }
+
+  pdl_launch();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------ host launchers
+cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                        const GemmArgs& args, int grid, bool pdl, cudaStream_t stream) {
+  static bool attr_set[3] = {false, false, false};
+  void (*fn)(CUtensorMap, CUtensorMap, GemmArgs) =
+      (epi == 1) ? moe_gemm_kernel<1> : moe_gemm_kernel<2>;
+  if (!attr_set[epi]) {
+    cudaError_t err = cudaFuncSetAttribute((const void*)fn,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kGemmSmemBytes);
+    if (err != cudaSuccess) return err;
+    attr_set[epi] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, args);
+}
+
+cudaError_t launch_requant_debug(const float* a, int rows, int cols, uint8_t* codes,
+                                 uint8_t* sbytes, cudaStream_t stream) {
+  long long nblk = (long long)rows * (cols / 32);
+  int grid = (int)((nblk + 255) / 256);
+  if (grid < 1) grid = 1;
+  if (grid > 4096) grid = 4096;
+  requant_debug_kernel<<<grid, 256, 0, stream>>>(a, rows, cols, codes, sbytes);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,101 @@
+// moe_internal.cuh -- shared definitions of the libmoe CUDA sources:
+// workspace layout, device status word, tile constants.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- constants
+constexpr int kBlockM = 128;        // rows per M tile (padding granule of the expert layout)
+constexpr int kBlockN = 256;        // weight rows per N tile
+constexpr int kBlockK = 128;        // K elements per pipeline stage (4 MMAs of K=32)
+constexpr int kSfChunk = 512;       // bytes of one 128-row x 4-K-block scale chunk
+constexpr int kPlanChunk = 1024;    // assignments per plan block
+constexpr int kMaxE = 1024;
+constexpr int kMaxTopk = 32;
+
+// header words at the start of the workspace
+enum HdrWord : int {
+  kHdrStatus = 0,     // moe_status of the last plan/forward (device side)
+  kHdrP = 1,          // padded rows P
+  kHdrMTiles = 2,     // P / kBlockM
+  kHdrBadIds = 3,     // number of skipped invalid expert ids
+  kHdrTimeoutSite = 4,
+  kHdrWords = 64
+};
+
+// byte offsets of every region of the workspace (all 1024-byte aligned)
+struct WsLayout {
+  size_t hdr, counts, offs, poffs, chunk, row_of, src_of, tile_expert;
+  size_t xp, xp_sf, a2, a2_sf, yp;
+  size_t total;
+  int R, P_max, MT_max, NCH;
+};
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Upper bound on padded rows over every routing: each non-empty expert adds
+// at most kBlockM-1 rows of padding, and at most min(E, R) experts are
+// non-empty.
+__host__ __device__ inline int max_padded_rows(int R, int E) {
+  long long nonempty = R < E ? R : E;
+  long long p = (long long)R + nonempty * (kBlockM - 1);
+  return (int)align_up((size_t)p, kBlockM);
+}
+
+inline WsLayout ws_layout(const moe_shape& s) {
+  WsLayout L{};
+  L.R = s.T * s.topk;
+  L.P_max = max_padded_rows(L.R, s.E);
+  L.MT_max = L.P_max / kBlockM;
+  L.NCH = (L.R + kPlanChunk - 1) / kPlanChunk;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  L.hdr = take(kHdrWords * 4);
+  L.counts = take((size_t)s.E * 4);
+  L.offs = take((size_t)(s.E + 1) * 4);
+  L.poffs = take((size_t)(s.E + 1) * 4);
+  L.chunk = take((size_t)L.NCH * s.E * 4);
+  L.row_of = take((size_t)L.R * 4);
+  L.src_of = take((size_t)L.P_max * 4);
+  L.tile_expert = take((size_t)L.MT_max * 4);
+  L.xp = take((size_t)L.P_max * s.H);
+  L.xp_sf = take((size_t)L.MT_max * (s.H / 128) * kSfChunk);
+  L.a2 = take((size_t)L.P_max * s.I);
+  L.a2_sf = take((size_t)L.MT_max * (s.I / 128) * kSfChunk);
+  L.yp = take((size_t)L.P_max * s.H * 4);
+  L.total = off;
+  return L;
+}
+
+// arguments of the grouped GEMM kernel (both linears)
+struct GemmArgs {
+  const uint8_t* sfa;      // activation scale chunks [MT][KB][512]
+  const uint8_t* sfb;      // weight scale chunks [E][KB][n_rows/128][512]
+  int* hdr;                // workspace header
+  const int* tile_expert;  // expert of every m-tile
+  const int* src_of;       // assignment of every padded row (-1 = padding)
+  int KB;                  // K / 128
+  int n_rows;              // weight rows per expert
+  int NT;                  // ceil(n_rows / 256)
+  uint8_t* a2;             // linear1 out: E4M3 [P, I]
+  uint8_t* a2_sf;          // linear1 out: scale chunks [MT][I/128][512]
+  int I;
+  float* yp;               // linear2 out: FP32 [P, H]
+  const float* topk_w;     // [T*k]
+  int H;
+};
+
+// record the first error of a call in the status word
+__device__ inline void set_status(int* hdr, int code) { atomicCAS(&hdr[kHdrStatus], 0, code); }
+
+}  // namespace moe

@@ -1,0 +1,308 @@
+// moe_kernels.cu -- the HBM-bound kernels of the MoE layer forward:
+//   plan    (routing bookkeeping: histogram, prefix sums, stable scatter),
+//   permute (dispatch: gather token rows and their scales into
+//            expert-contiguous order),
+//   combine (weighted top-k reduction of the FP32 partial rows into BF16),
+//   transform (one-time weight repack).
+// ("DeepSeek DeepGEMM 2026年4月重磅更新：Mega MoE融合算子、FP4精度与极致性能优化",
+//  section 3.1: the dispatch and combine steps around the two expert linears;
+//  section 3.3: transform_weights_for_mega_moe and the buffer fields.)
+#include <cuda_bf16.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+__device__ __forceinline__ void pdl_wait_k() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_k() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// byte offset of (row, K-group) inside scale chunks laid out [row/128][G][512]
+__device__ __forceinline__ size_t sf_chunk_offset(int row, int kg, int G) {
+  return ((size_t)(row >> 7) * G + kg) * kSfChunk + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+}
+
+// ------------------------------------------------------------------- plan
+// K1a: per-chunk expert histograms.  chunk_counts[b][e] = assignments of
+// chunk b (kPlanChunk consecutive flattened slots) routed to expert e.
+__global__ void plan_count_kernel(const int32_t* __restrict__ idx, int R, int E,
+                                  int* __restrict__ chunk_counts, int* __restrict__ hdr) {
+  extern __shared__ int hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int base = blockIdx.x * kPlanChunk;
+  int bad = 0;
+  for (int i = threadIdx.x; i < kPlanChunk && base + i < R; i += blockDim.x) {
+    const int e = idx[base + i];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    else if (e != -1) bad++;
+  }
+  if (bad) {
+    atomicAdd(&hdr[kHdrBadIds], bad);
+    set_status(hdr, MOE_ERR_BAD_EXPERT_ID);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// K1b (one block of 1024 threads): turn chunk histograms into per-chunk
+// starting ranks (exclusive, in place), expert counts, offsets, padded
+// offsets, the m-tile -> expert table and -1 for padding rows of src_of.
+__global__ void __launch_bounds__(1024) plan_scan_kernel(int E, int NCH, int* __restrict__ chunk_counts,
+                                                         int* __restrict__ counts,
+                                                         int* __restrict__ offs,
+                                                         int* __restrict__ poffs,
+                                                         int* __restrict__ tile_expert,
+                                                         int* __restrict__ src_of,
+                                                         int* __restrict__ hdr) {
+  __shared__ int warp_tot[2][32];
+  __shared__ int carry[2];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid == 0) carry[0] = carry[1] = 0;
+  __syncthreads();
+  for (int e0 = 0; e0 < E; e0 += 1024) {
+    const int e = e0 + tid;
+    int c = 0;
+    if (e < E) {
+      for (int b = 0; b < NCH; ++b) {
+        const int v = chunk_counts[(size_t)b * E + e];
+        chunk_counts[(size_t)b * E + e] = c;
+        c += v;
+      }
+      counts[e] = c;
+    }
+    const int pc = (c + kBlockM - 1) / kBlockM * kBlockM;
+    // block-wide inclusive scans of c and pc
+    int s0 = c, s1 = pc;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int t0 = __shfl_up_sync(0xffffffffu, s0, d), t1 = __shfl_up_sync(0xffffffffu, s1, d);
+      if (lane >= d) { s0 += t0; s1 += t1; }
+    }
+    if (lane == 31) { warp_tot[0][wid] = s0; warp_tot[1][wid] = s1; }
+    __syncthreads();
+    if (wid == 0) {
+      int w0 = warp_tot[0][lane], w1 = warp_tot[1][lane];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int t0 = __shfl_up_sync(0xffffffffu, w0, d), t1 = __shfl_up_sync(0xffffffffu, w1, d);
+        if (lane >= d) { w0 += t0; w1 += t1; }
+      }
+      warp_tot[0][lane] = w0;
+      warp_tot[1][lane] = w1;
+    }
+    __syncthreads();
+    const int pre0 = carry[0] + (wid ? warp_tot[0][wid - 1] : 0) + s0 - c;
+    const int pre1 = carry[1] + (wid ? warp_tot[1][wid - 1] : 0) + s1 - pc;
+    if (e < E) {
+      offs[e] = pre0;
+      poffs[e] = pre1;
+      for (int mt = pre1 / kBlockM; mt < (pre1 + pc) / kBlockM; ++mt) tile_expert[mt] = e;
+      for (int r = pre1 + c; r < pre1 + pc; ++r) src_of[r] = -1;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      carry[0] += warp_tot[0][31];
+      carry[1] += warp_tot[1][31];
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    offs[E] = carry[0];
+    poffs[E] = carry[1];
+    hdr[kHdrP] = carry[1];
+    hdr[kHdrMTiles] = carry[1] / kBlockM;
+  }
+}
+
+// K1c: stable scatter.  Thread i of block b owns assignment b*kPlanChunk+i;
+// its row is padded_offs[e] + (assignments of e in earlier chunks) +
+// (assignments of e in earlier warps of this chunk) + (earlier lanes of its
+// warp with the same expert), which orders each expert's rows by ascending
+// flattened index.
+__global__ void __launch_bounds__(1024) plan_scatter_kernel(const int32_t* __restrict__ idx, int R,
+                                                            int E,
+                                                            const int* __restrict__ chunk_base,
+                                                            const int* __restrict__ poffs,
+                                                            int* __restrict__ row_of,
+                                                            int* __restrict__ src_of) {
+  extern __shared__ unsigned short wcnt[];  // [32 warps][E]
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  const int a = blockIdx.x * kPlanChunk + tid;
+  int e = -1;
+  if (a < R) {
+    e = idx[a];
+    if (e < 0 || e >= E) e = -1;
+  }
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int rank_w = __popc(peers & ((1u << lane) - 1u));
+  if (e >= 0 && rank_w == 0) wcnt[wid * E + e] = (unsigned short)__popc(peers);
+  __syncthreads();
+  if (a < R) {
+    if (e < 0) {
+      row_of[a] = -1;
+    } else {
+      int rank = chunk_base[(size_t)blockIdx.x * E + e] + rank_w;
+      for (int w = 0; w < wid; ++w) rank += wcnt[w * E + e];
+      const int row = poffs[e] + rank;
+      row_of[a] = row;
+      src_of[row] = a;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- permute
+// One warp per padded row: copy x[t] (H bytes) into Xp[row] and its scale
+// words into the chunked layout the GEMM streams.  Padding rows are skipped.
+__global__ void permute_kernel(const uint8_t* __restrict__ x, const int32_t* __restrict__ x_sf,
+                               const int* __restrict__ src_of, const int* __restrict__ hdr, int H,
+                               int topk, uint8_t* __restrict__ xp, uint8_t* __restrict__ xp_sf) {
+  pdl_wait_k();
+  const int P = hdr[kHdrP];
+  const int lane = threadIdx.x & 31;
+  const int warps = (gridDim.x * blockDim.x) >> 5;
+  const int G = H / 128;
+  for (int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; row < P; row += warps) {
+    const int src = src_of[row];
+    if (src < 0) continue;
+    const int t = src / topk;
+    const uint4* s4 = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+    uint4* d4 = reinterpret_cast<uint4*>(xp + (size_t)row * H);
+    for (int i = lane; i < H / 16; i += 32) d4[i] = __ldg(&s4[i]);
+    for (int kg = lane; kg < G; kg += 32)
+      *reinterpret_cast<int32_t*>(xp_sf + sf_chunk_offset(row, kg, G)) = x_sf[(size_t)t * G + kg];
+  }
+  pdl_launch_k();
+}
+
+// ---------------------------------------------------------------- combine
+// y[t] = BF16_RNE( sum_s Yp[row_of[t][s]] ) in slot order, FP32 (the top-k
+// weight was applied by the linear2 epilogue).  One block per token.
+__global__ void combine_kernel(const float* __restrict__ yp, const int* __restrict__ row_of, int T,
+                               int H, int topk, __nv_bfloat16* __restrict__ y) {
+  pdl_wait_k();
+  __shared__ int rows[kMaxTopk];
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();
+    if (threadIdx.x < topk) rows[threadIdx.x] = row_of[(size_t)t * topk + threadIdx.x];
+    __syncthreads();
+    for (int c = threadIdx.x * 4; c < H; c += blockDim.x * 4) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; s < topk; ++s) {
+        const int r = rows[s];
+        if (r < 0) continue;
+        const float4 v = __ldg(reinterpret_cast<const float4*>(yp + (size_t)r * H + c));
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 packed;
+      packed.x = *reinterpret_cast<uint32_t*>(&lo);
+      packed.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(y + (size_t)t * H + c) = packed;
+    }
+  }
+  pdl_launch_k();
+}
+
+// -------------------------------------------------------------- transform
+// One thread per (expert, K-block, transformed row): 64 bytes of codes and
+// one 32-bit word of scales.  interleave != 0 applies the W1 gate/up
+// interleave: transformed row n' = 256g + j takes gate row 128g + j (j < 128)
+// or up row half + 128g + (j - 128).
+__global__ void transform_kernel(const uint8_t* __restrict__ w, const uint8_t* __restrict__ w_sf,
+                                 int E, int N, int K, int interleave, uint8_t* __restrict__ wt,
+                                 uint8_t* __restrict__ wt_sf) {
+  const int KB = K / 128;
+  const long long total = (long long)E * KB * N;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(i % N);
+    const int kb = (int)((i / N) % KB);
+    const int e = (int)(i / ((long long)N * KB));
+    int src_row = n;
+    if (interleave) {
+      const int g = n >> 8, j = n & 255;
+      src_row = (j < 128) ? (g * 128 + j) : (N / 2 + g * 128 + (j - 128));
+    }
+    const size_t srow = (size_t)e * N + src_row;
+    const uint4* s4 = reinterpret_cast<const uint4*>(w + srow * (K / 2) + (size_t)kb * 64);
+    uint4* d4 = reinterpret_cast<uint4*>(wt + (((size_t)e * KB + kb) * N + n) * 64);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) d4[v] = s4[v];
+    const uint32_t sfw = *reinterpret_cast<const uint32_t*>(w_sf + srow * (K / 32) + (size_t)kb * 4);
+    const size_t chunk = ((size_t)e * KB + kb) * (N / 128) + (n >> 7);
+    *reinterpret_cast<uint32_t*>(wt_sf + chunk * kSfChunk + (n & 31) * 16 + ((n >> 5) & 3) * 4) = sfw;
+  }
+}
+
+// ---------------------------------------------------------------- launchers
+static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem, bool pdl,
+                              cudaStream_t stream, void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int* chunk, int* counts,
+                        int* offs, int* poffs, int* tile_expert, int* row_of, int* src_of,
+                        int* hdr, cudaStream_t stream) {
+  static bool attr_set = false;
+  const size_t scatter_smem = (size_t)32 * E * sizeof(unsigned short);
+  if (!attr_set) {
+    cudaError_t err = cudaFuncSetAttribute((const void*)plan_scatter_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           32 * kMaxE * (int)sizeof(unsigned short));
+    if (err != cudaSuccess) return err;
+    attr_set = true;
+  }
+  if (R > 0) {
+    plan_count_kernel<<<NCH, 256, E * sizeof(int), stream>>>(idx, R, E, chunk, hdr);
+  }
+  plan_scan_kernel<<<1, 1024, 0, stream>>>(E, NCH, chunk, counts, offs, poffs, tile_expert, src_of,
+                                           hdr);
+  if (R > 0) {
+    plan_scatter_kernel<<<NCH, 1024, scatter_smem, stream>>>(idx, R, E, chunk, poffs, row_of,
+                                                             src_of);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const uint8_t* x, const int32_t* x_sf, const int* src_of,
+                           const int* hdr, int H, int topk, uint8_t* xp, uint8_t* xp_sf, int grid,
+                           bool pdl, cudaStream_t stream) {
+  void* args[] = {(void*)&x, (void*)&x_sf, (void*)&src_of, (void*)&hdr, (void*)&H,
+                  (void*)&topk, (void*)&xp, (void*)&xp_sf};
+  return launch_pdl((const void*)permute_kernel, dim3(grid), dim3(256), 0, pdl, stream, args);
+}
+
+cudaError_t launch_combine(const float* yp, const int* row_of, int T, int H, int topk, uint16_t* y,
+                           int grid, bool pdl, cudaStream_t stream) {
+  __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(y);
+  void* args[] = {(void*)&yp, (void*)&row_of, (void*)&T, (void*)&H, (void*)&topk, (void*)&yb};
+  int threads = H / 4 < 256 ? ((H / 4 + 31) / 32) * 32 : 256;
+  return launch_pdl((const void*)combine_kernel, dim3(grid), dim3(threads), 0, pdl, stream, args);
+}
+
+cudaError_t launch_transform(const uint8_t* w, const uint8_t* w_sf, int E, int N, int K,
+                             int interleave, uint8_t* wt, uint8_t* wt_sf, cudaStream_t stream) {
+  const long long total = (long long)E * (K / 128) * N;
+  long long grid = (total + 255) / 256;
+  if (grid > 65535LL * 16) grid = 65535LL * 16;
+  if (grid < 1) grid = 1;
+  transform_kernel<<<(unsigned)grid, 256, 0, stream>>>(w, w_sf, E, N, K, interleave, wt, wt_sf);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,203 @@
+/*
+ * moe.h -- C ABI of libmoe: one FP8 x FP4 Mixture-of-Experts layer forward
+ * on a single NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes.  The MoE forward named in
+ *   "DeepSeek DeepGEMM 2026年4月重磅更新：Mega MoE融合算子、FP4精度与极致性能优化"
+ *   (chenxutan.com), section 3.1 and 3.2 (dispatch -> linear1 (FP8xFP4) ->
+ *   SwiGLU -> linear2 (FP8xFP4) -> combine, fused), section 3.3 (the call's
+ *   inputs: x (FP8), x_sf, topk_idx, topk_weights, weights l1 / l2 in FP4 with
+ *   UE8M0 scale factors, a caller-allocated BF16 y) and section 4.2 (UE8M0
+ *   scale factors packed four per 32-bit int, FP32 accumulation);
+ *   "DeepGEMM: DeepSeek 把大模型核心算子打包成一座 CUDA 训练场"
+ *   (zevenfang.github.io), section 4 (SM100 consumes packed UE8M0 scales)
+ *   and section 5 (the five fused steps).
+ * On one GPU, dispatch is an on-device permutation of token rows into
+ * expert-contiguous order and combine is an on-device weighted reduction.
+ *
+ * For every token t and slot s with e = topk_idx[t][s] != -1:
+ *   g   = W1[e] . x[t]                       (2I outputs; rows [0,I) gate, [I,2I) up)
+ *   a   = silu(g[0:I]) * g[I:2I]             (FP32; silu(z) = z / (1 + exp(-z)))
+ *   a'  = E4M3 requantisation of a, one UE8M0 scale per 32 consecutive values,
+ *         scale exponent = smallest e with 448 * 2^e >= amax (0 for amax 0)
+ *   o   = W2[e] . a'                         (H outputs)
+ *   y[t] = BF16_RNE( sum over s in slot order of topk_w[t][s] * o )   (FP32 sum)
+ * All products are block-scaled: every 1x32 block along K of x, W1, W2 and a'
+ * carries one UE8M0 scale (value 2^(b-127)).
+ *
+ * Canonical layouts (row-major, little-endian):
+ *   x        uint8  [T, H]        E4M3 codes (OCP e4m3fn: bias 7, max 448, no Inf)
+ *   x_sf     int32  [T, H/128]    byte j of word i = UE8M0 scale of K-block 4i+j
+ *   topk_idx int32  [T, k]        expert ids; -1 = unused slot
+ *   topk_w   fp32   [T, k]
+ *   w1       uint8  [E, 2I, H/2]  E2M1 codes, two per byte, low nibble = even k
+ *   w1_sf    uint8  [E, 2I, H/32] UE8M0 per 1x32 block
+ *   w2       uint8  [E, H, I/2],  w2_sf uint8 [E, H, I/32]
+ *   y        uint16 [T, H]        BF16 bits
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are DEVICE pointers owned by the caller unless the parameter
+ *     says "host".  The library never allocates device memory and never
+ *     frees anything it did not allocate.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns an error status and launches nothing.
+ *   - moe_plan and moe_forward enqueue work on `stream` and return without
+ *     synchronising; data-dependent problems (an expert id outside
+ *     [-1, E), a device wait that timed out) are recorded in a status word
+ *     inside the workspace and read back by moe_get_device_status.
+ *   - A workspace is used by one call sequence at a time; calls that share a
+ *     workspace must be ordered on one stream.
+ *   - Supported shapes: H % 128 == 0, I % 128 == 0, 1 <= k <= 32,
+ *     1 <= E <= 1024, 0 <= T, T * k <= 2^24.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,      /* null pointer, misaligned pointer, negative size */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,/* shape outside the supported set above */
+  MOE_ERR_WORKSPACE = 3,        /* workspace too small */
+  MOE_ERR_CUDA = 4,             /* a CUDA runtime / driver call failed */
+  MOE_ERR_TIMEOUT = 5,          /* device status: a bounded device wait expired */
+  MOE_ERR_BAD_EXPERT_ID = 6     /* device status: an id outside [-1, E) was skipped */
+} moe_status;
+
+typedef struct {
+  int T;    /* tokens */
+  int H;    /* hidden size (K of linear1, N of linear2) */
+  int I;    /* intermediate size after SwiGLU (linear1 has 2I outputs) */
+  int E;    /* experts */
+  int topk; /* experts per token */
+} moe_shape;
+
+/* Human-readable name of a status code (static storage). */
+const char* moe_status_string(moe_status s);
+
+/* Row granularity of the padded expert-contiguous layout (rows of one
+ * expert start at a multiple of this).  Returns 128. */
+int moe_block_m(void);
+
+/* Cap on the number of SMs used by the persistent kernels (0 = all SMs).
+ * "DeepSeek DeepGEMM 2026年4月重磅更新" section 9.2 (set_num_sms).
+ * Process-wide; takes effect for calls enqueued afterwards. */
+void moe_set_num_sms(int num_sms);
+
+/* Enable (1) or disable (0) programmatic dependent launch between the
+ * kernels of one forward.  "DeepSeek DeepGEMM 2026年4月重磅更新" section 6
+ * (PDL moves kernel-to-kernel dependencies onto the GPU).  Default 1. */
+void moe_set_pdl(int enable);
+
+/* ---------------------------------------------------------------- weights */
+/* Bytes of one transformed weight: which = 1 for W1, 2 for W2.  Returns the
+ * FP4 byte count and writes the scale-factor byte count to *sf_bytes (may
+ * be NULL).  Returns 0 for an unsupported shape. */
+size_t moe_transformed_bytes(const moe_shape* shape, int which, size_t* sf_bytes);
+
+/* One-time weight transform into the layout the GEMM kernels stream
+ * ("DeepSeek DeepGEMM 2026年4月重磅更新" section 3.3,
+ * transform_weights_for_mega_moe, FP4 + UE8M0 SF):
+ *   - W1 rows are interleaved in 128-row granules (gate rows 128g..128g+127
+ *     then up rows I+128g..I+128g+127) so that one 256-row tile holds the
+ *     gate and up rows of the same 128 SwiGLU outputs;
+ *   - FP4 codes are regrouped K-block-major: [E][K/128][rows][64 bytes], so
+ *     that each tile of one K-block is one contiguous run of memory (the
+ *     128-byte shared-memory swizzle is applied by the tensor-memory
+ *     accelerator on load);
+ *   - UE8M0 scales are regrouped into 512-byte chunks [E][K/128][rows/128]
+ *     of 128 rows x 4 K-blocks; byte (r%32)*16 + (r/32)*4 + j of a chunk is
+ *     row r, K-block j (four UE8M0 per 32-bit word).
+ * Inputs are the canonical w1 / w1_sf / w2 / w2_sf (device).  Outputs need
+ * moe_transformed_bytes() bytes each, 256-byte aligned, and must not alias
+ * the inputs.  Enqueued on `stream`. */
+moe_status moe_transform_weights(const moe_shape* shape, const uint8_t* w1, const uint8_t* w1_sf,
+                                 const uint8_t* w2, const uint8_t* w2_sf, void* w1_t,
+                                 void* w1_sf_t, void* w2_t, void* w2_sf_t, moe_stream_t stream);
+
+/* -------------------------------------------------------------- workspace */
+/* Bytes of workspace one forward needs for this shape: the plan, the
+ * permuted activations and their scales, the requantised intermediate and
+ * its scales, and the FP32 weighted partial outputs.  It is an upper bound
+ * over every possible routing (rows padded per expert to moe_block_m()). */
+size_t moe_workspace_bytes(const moe_shape* shape);
+
+/* ------------------------------------------------------------------- plan */
+/* Routing plan (the dispatch bookkeeping of "DeepSeek DeepGEMM 2026年4月重磅
+ * 更新" section 3.1): per-expert histogram of topk_idx, exclusive prefix sum,
+ * padded offsets (multiples of moe_block_m()), the row of every assignment
+ * (rows of one expert ordered by ascending t*k+s) and the tile schedule.
+ * topk_idx: device int32 [T, k].  workspace: device, 256-byte aligned,
+ * at least moe_workspace_bytes(shape) bytes.  Resets the device status word.
+ * Enqueued on `stream`; nothing is synchronised. */
+moe_status moe_plan(const moe_shape* shape, const int32_t* topk_idx, void* workspace,
+                    size_t ws_bytes, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- forward */
+/* The layer forward, using the plan already in `workspace` (moe_plan must be
+ * enqueued before it on the same stream with the same topk_idx):
+ * permute -> grouped GEMM1 + SwiGLU + E4M3 requant -> grouped GEMM2 x topk_w
+ * -> per-token combine into BF16.  x, x_sf, topk_w in canonical layout;
+ * w1_t / w1_sf_t / w2_t / w2_sf_t from moe_transform_weights; y: device
+ * uint16 [T, H] written completely.  All device pointers 16-byte aligned
+ * (transformed weights and workspace 256-byte aligned).  Enqueued on
+ * `stream`; nothing is synchronised. */
+moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* x_sf,
+                       const int32_t* topk_idx, const float* topk_w, const void* w1_t,
+                       const void* w1_sf_t, const void* w2_t, const void* w2_sf_t, uint16_t* y,
+                       void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* Host-buffer variant for callers whose activations live in host memory:
+ * copies x / x_sf / topk_idx / topk_w (HOST, preferably pinned) to the
+ * device staging area at the end of `workspace`, runs moe_plan and
+ * moe_forward, copies y back to `y_host` (HOST) and synchronises `stream`.
+ * Needs moe_workspace_bytes_host(shape) bytes of workspace. */
+size_t moe_workspace_bytes_host(const moe_shape* shape);
+moe_status moe_forward_host(const moe_shape* shape, const uint8_t* x_host,
+                            const int32_t* x_sf_host, const int32_t* topk_idx_host,
+                            const float* topk_w_host, const void* w1_t, const void* w1_sf_t,
+                            const void* w2_t, const void* w2_sf_t, uint16_t* y_host,
+                            void* workspace, size_t ws_bytes, moe_stream_t stream);
+
+/* ------------------------------------------------------------- diagnostics */
+/* Synchronises `stream` and returns the device status word of the last
+ * plan / forward that used `workspace` (MOE_OK, MOE_ERR_BAD_EXPERT_ID or
+ * MOE_ERR_TIMEOUT), or MOE_ERR_CUDA if the stream itself failed. */
+moe_status moe_get_device_status(const void* workspace, moe_stream_t stream);
+
+/* Copies the plan out of `workspace` for bit-exact checking (synchronises
+ * `stream`).  All outputs are HOST buffers: counts [E], offs [E+1],
+ * padded_offs [E+1], row_of [T*k] (-1 for skipped slots), src_of [P] where
+ * P = padded_offs[E] (-1 for padding rows); *P_out receives P.  src_of may be
+ * NULL; otherwise it must hold moe_plan_max_rows(shape) entries. */
+int moe_plan_max_rows(const moe_shape* shape);
+moe_status moe_plan_export(const moe_shape* shape, const void* workspace, int32_t* counts,
+                           int32_t* offs, int32_t* padded_offs, int32_t* row_of, int32_t* src_of,
+                           int32_t* P_out, moe_stream_t stream);
+
+/* Kernel timing: when `events` is not NULL and n >= 5, every following
+ * moe_forward records events[0..4] (cudaEvent_t handles owned by the
+ * caller) on its stream: before the permute kernel, after it, after the
+ * linear1 kernel, after the linear2 kernel and after the combine kernel.
+ * NULL stops it.  Process-wide; the handles must outlive their use. */
+void moe_set_timing_events(void* const* events, int n);
+
+/* Test hook: runs the GEMM1 epilogue's requantiser on `a` (device fp32
+ * [rows, cols], cols % 32 == 0) and writes E4M3 codes (device uint8
+ * [rows, cols]) and UE8M0 bytes (device uint8 [rows, cols/32]).  Same
+ * device code as the fused epilogue. */
+moe_status moe_debug_requant(const float* a, int rows, int cols, uint8_t* codes, uint8_t* sbytes,
+                             moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

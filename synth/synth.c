@@ -14,8 +14,9 @@
  * Random numbers: counter-based.  Draw i of (seed, stream) is the splitmix64
  * finaliser applied to (seed ^ stream << 40 ^ i) + 0x9E3779B97F4A7C15; two
  * 53-bit uniforms make one Box-Muller pair (cos branch for even i, sin for
- * odd i).  Streams: 1 = x, 2 = W1, 3 = W2, 4 = router logits, 5 = the
- * random expert ranking behind the Zipf bias.
+ * odd i; computed in single precision).  Streams: 1 = x, 2 = W1,
+ * 3 = W2, 4 = router logits, 5 = the random expert ranking behind the
+ * Zipf bias.
  */
 #include <math.h>
 #include <stdint.h>
@@ -39,11 +40,13 @@ static inline double draw_unif(uint64_t seed, uint64_t stream, uint64_t i) {
 /* normals n[2p], n[2p+1] of (seed, stream) */
 static inline void draw_normal_pair(uint64_t seed, uint64_t stream, uint64_t p, double* n0,
                                     double* n1) {
-  double u1 = draw_unif(seed, stream, 2 * p), u2 = draw_unif(seed, stream, 2 * p + 1);
-  double r = sqrt(-2.0 * log(u1));
-  double th = TWO_PI * u2;
-  *n0 = r * cos(th);
-  *n1 = r * sin(th);
+  /* single-precision transcendental functions: ample for synthetic data */
+  float u1 = (float)draw_unif(seed, stream, 2 * p), u2 = (float)draw_unif(seed, stream, 2 * p + 1);
+  if (u1 <= 0.0f) u1 = 0x1.0p-30f;
+  float r = sqrtf(-2.0f * logf(u1));
+  float th = (float)TWO_PI * u2;
+  *n0 = (double)(r * cosf(th));
+  *n1 = (double)(r * sinf(th));
 }
 
 static inline double draw_normal(uint64_t seed, uint64_t stream, uint64_t i) {
@@ -110,8 +113,9 @@ void synth_x(int T, int H, uint64_t seed, uint8_t* x, int32_t* x_sf) {
       double amax = 0;
       for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(v[i]));
       int e = cast_exponent(amax, 448.0);
+      const double inv = ldexp(1.0, -e);         /* exact power of two */
       for (int i = 0; i < 32; ++i) {
-        double a = ldexp(v[i], -e);
+        double a = v[i] * inv;
         int c = nearest_code(g_e4m3_mag, 127, fabs(a));
         x[base + i] = (uint8_t)(c | (a < 0 ? 0x80 : 0));
       }
@@ -141,9 +145,10 @@ void synth_w(int E, int N, int K, uint64_t seed, uint64_t stream, double std, ui
       double amax = 0;
       for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(v[i]));
       int e = cast_exponent(amax, 6.0);
+      const double inv = ldexp(1.0, -e);         /* exact power of two */
       uint8_t* dst = w + (size_t)r * (K / 2) + (size_t)b * 16;
       for (int i = 0; i < 32; i += 2) {
-        double a0 = ldexp(v[i], -e), a1 = ldexp(v[i + 1], -e);
+        double a0 = v[i] * inv, a1 = v[i + 1] * inv;
         int c0 = nearest_code(g_e2m1_mag, 8, fabs(a0)) | (a0 < 0 ? 8 : 0);
         int c1 = nearest_code(g_e2m1_mag, 8, fabs(a1)) | (a1 < 0 ? 8 : 0);
         dst[i / 2] = (uint8_t)(c0 | (c1 << 4));
