@@ -9,7 +9,8 @@
 
 namespace moe {
 cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                        const GemmArgs& args, int grid, bool pdl, cudaStream_t stream);
+                        const CUtensorMap& tmOut, const GemmArgs& args, int grid, bool pdl,
+                        cudaStream_t stream);
 cudaError_t launch_requant_debug(const float* a, int rows, int cols, uint8_t* codes,
                                  uint8_t* sbytes, cudaStream_t stream);
 cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int* chunk, int* counts,
@@ -100,6 +101,19 @@ bool encode_wgt(CUtensorMap* m, const void* base, int E, int KB, int n_rows) {
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(base), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// FP32 partial rows [rows, N]: TMA store box 16 columns x 32 rows, 64-byte swizzle
+bool encode_out_f32(CUtensorMap* m, const void* base, int rows, int N) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+  cuuint32_t box[2] = {16, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -260,11 +274,12 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   const int KB1 = sh.H / 128, KB2 = sh.I / 128;
   const int NT1 = (2 * sh.I + kBlockN - 1) / kBlockN, NT2 = (sh.H + kBlockN - 1) / kBlockN;
 
-  CUtensorMap tmX, tmW1, tmA2, tmW2;
+  CUtensorMap tmX, tmW1, tmA2, tmW2, tmYp;
   if (!encode_act(&tmX, ws.xp(), ws.L.P_max, sh.H) ||
       !encode_wgt(&tmW1, w1_t, sh.E, KB1, 2 * sh.I) ||
       !encode_act(&tmA2, ws.a2(), ws.L.P_max, sh.I) ||
-      !encode_wgt(&tmW2, w2_t, sh.E, KB2, sh.H))
+      !encode_wgt(&tmW2, w2_t, sh.E, KB2, sh.H) ||
+      !encode_out_f32(&tmYp, ws.yp(), ws.L.P_max, sh.H))
     return MOE_ERR_CUDA;
 
   // dispatch: permute rows into expert-contiguous order
@@ -293,7 +308,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   long long tiles1 = (long long)ws.L.MT_max * NT1;
   int grid1 = (int)(tiles1 < sms ? tiles1 : sms);
   if (grid1 < 1) grid1 = 1;
-  e = launch_gemm(1, tmX, tmW1, g1, grid1, pdl, s);
+  e = launch_gemm(1, tmX, tmW1, tmYp, g1, grid1, pdl, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   record_event(2, s);
 
@@ -308,7 +323,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   long long tiles2 = (long long)ws.L.MT_max * NT2;
   int grid2 = (int)(tiles2 < sms ? tiles2 : sms);
   if (grid2 < 1) grid2 = 1;
-  e = launch_gemm(2, tmA2, tmW2, g2, grid2, pdl, s);
+  e = launch_gemm(2, tmA2, tmW2, tmYp, g2, grid2, pdl, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   record_event(3, s);
 

@@ -41,8 +41,9 @@ constexpr int kGemmThreads = 64 + 32 * kNumEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;    // FP32 accumulator, 256 columns
 constexpr uint32_t kSfCol = 256;   // scale buffers: buf b -> SFA at +16b (4 cols), SFB at +16b+4 (8)
-constexpr size_t kGemmSmemBytes =
-    1024 + (size_t)kStages * (kSmemA + kSmemB + kSmemSFA + kSmemSFB) + 256;
+constexpr int kOutStage = 2048;      // per epilogue warp: 32 rows x 16 FP32, 64-byte swizzle
+constexpr size_t kGemmSmemBytes = 1024 + (size_t)kStages * (kSmemA + kSmemB + kSmemSFA + kSmemSFB) +
+                                  (size_t)kNumEpiWarps * kOutStage + 256;
 
 // ------------------------------------------------------------- requantiser
 // Smallest e with 448 * 2^e >= amax, from the bits of amax (448 = 1.75 * 2^8):
@@ -107,7 +108,8 @@ __device__ __forceinline__ void pdl_launch() {
 template <int kEpi>  // 1: SwiGLU + requant (linear1), 2: x topk_w, FP32 rows (linear2)
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                    const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+                    const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmOut, const GemmArgs args) {
   using namespace ptx;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<size_t>(smem_raw), 1024));
@@ -115,7 +117,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* sB = sA + kStages * kSmemA;
   uint8_t* sSFA = sB + kStages * kSmemB;
   uint8_t* sSFB = sSFA + kStages * kSmemSFA;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + kStages * kSmemSFB);
+  uint8_t* sOut = sSFB + kStages * kSmemSFB;  // epilogue staging, 1024-aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kNumEpiWarps * kOutStage);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 1;
@@ -138,6 +141,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (kEpi == 2) prefetch_tmap(&tmOut);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, kTmemCols);
@@ -285,8 +289,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
       const int row = mt * kBlockM + r;
       const int src = args.src_of[row];
-      if (src < 0) continue;  // padding row (the loop head reconverges the warp)
       if (kEpi == 1) {
+        if (src < 0) continue;  // padding row (the loop head reconverges the warp)
         uint32_t sbytes = 0;
         uint8_t* dst = args.a2 + (size_t)row * args.I + nt * 128 + 64 * h;
 #pragma unroll
@@ -296,7 +300,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int i = 0; i < 32; ++i) {
             const float g = __uint_as_float(v[b][i]);
             const float u = __uint_as_float(v[2 + b][i]);
-            a[i] = g / (1.0f + __expf(-g)) * u;
+            a[i] = g * __frcp_rn(1.0f + __expf(-g)) * u;  // silu(g) * u
           }
           uint32_t packed[8], sb;
           requant32(a, packed, sb);
@@ -309,20 +313,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                          (r & 31) * 16 + (r >> 5) * 4 + 2 * h;
         *reinterpret_cast<uint16_t*>(sfdst) = (uint16_t)sbytes;
       } else {
+        // weighted FP32 rows, written through shared memory by TMA stores:
+        // 8 chunks of 32 rows x 16 columns per warp (64-byte swizzled staging)
         const int col0 = nt * kBlockN + 128 * h;
-        if (col0 >= n_rows) continue;  // half tile at the end of N
-        const float w = args.topk_w[src];
-        float4* dst = reinterpret_cast<float4*>(args.yp + (size_t)row * args.H + col0);
+        if (col0 >= n_rows) continue;  // half tile at the end of N (warp-uniform)
+        const float w = src >= 0 ? args.topk_w[src] : 0.0f;
+        uint8_t* stg = sOut + ew * kOutStage;
+        const uint32_t stg_row = smem_u32(stg) + (uint32_t)lane * 64u;
+        const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 8; ++c) {
+          if (lane == 0) bulk_wait_group_read0();  // staging free again
+          __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[c * 8 + j] = make_float4(w * __uint_as_float(v[c][4 * j]),
-                                         w * __uint_as_float(v[c][4 * j + 1]),
-                                         w * __uint_as_float(v[c][4 * j + 2]),
-                                         w * __uint_as_float(v[c][4 * j + 3]));
+          for (int j = 0; j < 4; ++j) {
+            const int i0 = (c * 16 + j * 4) & 31, vb = (c * 16 + j * 4) >> 5;
+            st_shared_v4(stg_row + 16u * ((uint32_t)j ^ swz), w * __uint_as_float(v[vb][i0]),
+                         w * __uint_as_float(v[vb][i0 + 1]), w * __uint_as_float(v[vb][i0 + 2]),
+                         w * __uint_as_float(v[vb][i0 + 3]));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmOut, stg, col0 + 16 * c, mt * kBlockM + q * 32);
+            bulk_commit_group();
+          }
+        }
       }
     }
+    if (kEpi == 2 && lane == 0) bulk_wait_group0();  // stores complete before the CTA exits
   }
 
   pdl_launch();
@@ -337,9 +356,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ------------------------------------------------------------ host launchers
 cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                        const GemmArgs& args, int grid, bool pdl, cudaStream_t stream) {
+                        const CUtensorMap& tmOut, const GemmArgs& args, int grid, bool pdl,
+                        cudaStream_t stream) {
   static bool attr_set[3] = {false, false, false};
-  void (*fn)(CUtensorMap, CUtensorMap, GemmArgs) =
+  void (*fn)(CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs) =
       (epi == 1) ? moe_gemm_kernel<1> : moe_gemm_kernel<2>;
   if (!attr_set[epi]) {
     cudaError_t err = cudaFuncSetAttribute((const void*)fn,
@@ -358,7 +378,7 @@ cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, args);
+  return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, tmOut, args);
 }
 
 cudaError_t launch_requant_debug(const float* a, int rows, int cols, uint8_t* codes,
