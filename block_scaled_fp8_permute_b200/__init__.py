@@ -49,6 +49,7 @@ _SIGS = {
     "moe_block_m": (_i, []),
     "moe_set_num_sms": (None, [_i]),
     "moe_set_pdl": (None, [_i]),
+    "moe_set_gemm_variant": (None, [_i]),
     "moe_transformed_bytes": (_sz, [_shp, _i, ctypes.POINTER(_sz)]),
     "moe_transform_weights": (_i, [_shp] + [_vp] * 8 + [_vp]),
     "moe_workspace_bytes": (_sz, [_shp]),
@@ -117,6 +118,10 @@ def moe_set_num_sms(n: int) -> None:
 
 def moe_set_pdl(enable: bool) -> None:
     _lib.moe_set_pdl(1 if enable else 0)
+
+
+def moe_set_gemm_variant(variant: int) -> None:
+    _lib.moe_set_gemm_variant(variant)
 
 
 def moe_transformed_bytes(shp: MoeShape, which: int):

@@ -11,11 +11,15 @@ namespace moe {
 cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmOut, const GemmArgs& args, int grid, bool pdl,
                         cudaStream_t stream);
+cudaError_t launch_gemm_pair(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                             const CUtensorMap& tmSFA, const CUtensorMap& tmSFB,
+                             const CUtensorMap& tmOut, const GemmArgs& args, int num_pairs_grid,
+                             bool pdl, cudaStream_t stream);
 cudaError_t launch_requant_debug(const float* a, int rows, int cols, uint8_t* codes,
                                  uint8_t* sbytes, cudaStream_t stream);
 cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int* chunk, int* counts,
-                        int* offs, int* poffs, int* tile_expert, int* row_of, int* src_of,
-                        int* hdr, cudaStream_t stream);
+                        int* offs, int* poffs, int* tile_expert, int* mpair, int* row_of,
+                        int* src_of, int* hdr, cudaStream_t stream);
 cudaError_t launch_permute(const uint8_t* x, const int32_t* x_sf, const int* src_of,
                            const int* hdr, int H, int topk, uint8_t* xp, uint8_t* xp_sf, int grid,
                            bool pdl, cudaStream_t stream);
@@ -28,6 +32,7 @@ namespace {
 
 std::atomic<int> g_num_sms_cap{0};
 std::atomic<int> g_pdl{1};
+std::atomic<int> g_gemm_variant{0};
 std::mutex g_ev_mu;
 cudaEvent_t g_events[5];
 bool g_events_on = false;
@@ -90,14 +95,14 @@ bool encode_act(CUtensorMap* m, const void* base, int rows, int K) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// transformed weights [E*KB][n_rows][128 E2M1 = 64 bytes]: box 128 x 256 x 1;
+// transformed weights [E*KB][n_rows][128 E2M1 = 64 bytes]: box 128 x box_rows x 1;
 // the TMA unpacks every 16 codes (8 bytes) into a 16-byte shared-memory slot.
-bool encode_wgt(CUtensorMap* m, const void* base, int E, int KB, int n_rows) {
+bool encode_wgt(CUtensorMap* m, const void* base, int E, int KB, int n_rows, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {128, (cuuint64_t)n_rows, (cuuint64_t)E * KB};
   cuuint64_t strides[2] = {64, (cuuint64_t)n_rows * 64};
-  cuuint32_t box[3] = {128, 256, 1};
+  cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(base), dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -117,6 +122,20 @@ bool encode_out_f32(CUtensorMap* m, const void* base, int rows, int N) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// scale chunks [nchunks][512 bytes] as uint32 [nchunks][128]: box of
+// `chunks` consecutive chunks
+bool encode_sf(CUtensorMap* m, const void* base, long long nchunks, int chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, (cuuint64_t)nchunks};
+  cuuint64_t strides[1] = {512};
+  cuuint32_t box[2] = {128, (cuuint32_t)chunks};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Ws {
   WsLayout L;
   uint8_t* base;
@@ -128,6 +147,7 @@ struct Ws {
   int* row_of() const { return reinterpret_cast<int*>(base + L.row_of); }
   int* src_of() const { return reinterpret_cast<int*>(base + L.src_of); }
   int* tile_expert() const { return reinterpret_cast<int*>(base + L.tile_expert); }
+  int* mpair() const { return reinterpret_cast<int*>(base + L.mpair); }
   uint8_t* xp() const { return base + L.xp; }
   uint8_t* xp_sf() const { return base + L.xp_sf; }
   uint8_t* a2() const { return base + L.a2; }
@@ -183,6 +203,8 @@ int moe_block_m(void) { return kBlockM; }
 void moe_set_num_sms(int num_sms) { g_num_sms_cap.store(num_sms > 0 ? num_sms : 0); }
 
 void moe_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
+
+void moe_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }
 
 void moe_set_timing_events(void* const* events, int n) {
   std::lock_guard<std::mutex> lk(g_ev_mu);
@@ -244,7 +266,8 @@ moe_status moe_plan(const moe_shape* shape, const int32_t* topk_idx, void* works
   cudaError_t e = cudaMemsetAsync(ws.hdr(), 0, kHdrWords * 4, s);
   if (e == cudaSuccess)
     e = launch_plan(topk_idx, ws.L.R, shape->E, ws.L.NCH, ws.chunk(), ws.counts(), ws.offs(),
-                    ws.poffs(), ws.tile_expert(), ws.row_of(), ws.src_of(), ws.hdr(), s);
+                    ws.poffs(), ws.tile_expert(), ws.mpair(), ws.row_of(), ws.src_of(), ws.hdr(),
+                    s);
   return cuda_status(e);
 }
 
@@ -274,12 +297,20 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   const int KB1 = sh.H / 128, KB2 = sh.I / 128;
   const int NT1 = (2 * sh.I + kBlockN - 1) / kBlockN, NT2 = (sh.H + kBlockN - 1) / kBlockN;
 
-  CUtensorMap tmX, tmW1, tmA2, tmW2, tmYp;
+  // SM-pair tiles (variant 1) for linear1 (2I is a multiple of 256) and for
+  // linear2 when H is; one-SM tiles otherwise (and for 128-column tail tiles)
+  const bool pair1 = g_gemm_variant.load() == 1;
+  const bool pair2 = pair1 && (sh.H % 256) == 0;
+  CUtensorMap tmX, tmW1, tmA2, tmW2, tmYp, tmXsf, tmW1sf, tmA2sf, tmW2sf;
   if (!encode_act(&tmX, ws.xp(), ws.L.P_max, sh.H) ||
-      !encode_wgt(&tmW1, w1_t, sh.E, KB1, 2 * sh.I) ||
+      !encode_wgt(&tmW1, w1_t, sh.E, KB1, 2 * sh.I, pair1 ? 128 : 256) ||
       !encode_act(&tmA2, ws.a2(), ws.L.P_max, sh.I) ||
-      !encode_wgt(&tmW2, w2_t, sh.E, KB2, sh.H) ||
-      !encode_out_f32(&tmYp, ws.yp(), ws.L.P_max, sh.H))
+      !encode_wgt(&tmW2, w2_t, sh.E, KB2, sh.H, pair2 ? 128 : 256) ||
+      !encode_out_f32(&tmYp, ws.yp(), ws.L.P_max, sh.H) ||
+      !encode_sf(&tmXsf, ws.xp_sf(), (long long)ws.L.MT_max * KB1, 1) ||
+      !encode_sf(&tmW1sf, w1_sf_t, (long long)sh.E * KB1 * (2 * sh.I / 128), 2) ||
+      !encode_sf(&tmA2sf, ws.a2_sf(), (long long)ws.L.MT_max * KB2, 1) ||
+      (pair2 && !encode_sf(&tmW2sf, w2_sf_t, (long long)sh.E * KB2 * (sh.H / 128), 2)))
     return MOE_ERR_CUDA;
 
   // dispatch: permute rows into expert-contiguous order
@@ -292,12 +323,14 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   record_event(1, s);
 
+  const int max_pairs_grid = sms / 2 > 0 ? sms / 2 : 1;
   GemmArgs g1{};
   g1.sfa = ws.xp_sf();
   g1.sfb = static_cast<const uint8_t*>(w1_sf_t);
   g1.hdr = ws.hdr();
   g1.tile_expert = ws.tile_expert();
   g1.src_of = ws.src_of();
+  g1.mpair = ws.mpair();
   g1.KB = KB1;
   g1.n_rows = 2 * sh.I;
   g1.NT = NT1;
@@ -305,10 +338,15 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   g1.a2_sf = ws.a2_sf();
   g1.I = sh.I;
   g1.H = sh.H;
-  long long tiles1 = (long long)ws.L.MT_max * NT1;
-  int grid1 = (int)(tiles1 < sms ? tiles1 : sms);
-  if (grid1 < 1) grid1 = 1;
-  e = launch_gemm(1, tmX, tmW1, tmYp, g1, grid1, pdl, s);
+  if (pair1) {
+    long long work = (long long)ws.L.MP_max * NT1;
+    int pairs = (int)(work < max_pairs_grid ? work : max_pairs_grid);
+    e = launch_gemm_pair(1, tmX, tmW1, tmXsf, tmW1sf, tmYp, g1, pairs < 1 ? 1 : pairs, pdl, s);
+  } else {
+    long long tiles1 = (long long)ws.L.MT_max * NT1;
+    int grid1 = (int)(tiles1 < sms ? tiles1 : sms);
+    e = launch_gemm(1, tmX, tmW1, tmYp, g1, grid1 < 1 ? 1 : grid1, pdl, s);
+  }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   record_event(2, s);
 
@@ -320,10 +358,15 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   g2.NT = NT2;
   g2.yp = ws.yp();
   g2.topk_w = topk_w;
-  long long tiles2 = (long long)ws.L.MT_max * NT2;
-  int grid2 = (int)(tiles2 < sms ? tiles2 : sms);
-  if (grid2 < 1) grid2 = 1;
-  e = launch_gemm(2, tmA2, tmW2, tmYp, g2, grid2, pdl, s);
+  if (pair2) {
+    long long work = (long long)ws.L.MP_max * NT2;
+    int pairs = (int)(work < max_pairs_grid ? work : max_pairs_grid);
+    e = launch_gemm_pair(2, tmA2, tmW2, tmA2sf, tmW2sf, tmYp, g2, pairs < 1 ? 1 : pairs, pdl, s);
+  } else {
+    long long tiles2 = (long long)ws.L.MT_max * NT2;
+    int grid2 = (int)(tiles2 < sms ? tiles2 : sms);
+    e = launch_gemm(2, tmA2, tmW2, tmYp, g2, grid2 < 1 ? 1 : grid2, pdl, s);
+  }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   record_event(3, s);
 

@@ -1,0 +1,98 @@
+// moe_epilogue.cuh -- the two fused GEMM epilogues, shared by the one-SM and
+// the SM-pair grouped GEMM kernels.  One thread owns one accumulator row
+// (TMEM lane) and one 128-column half of the 256-column tile.
+//   linear1 (kEpi 1): columns [0,128) of the tile are gate outputs, [128,256)
+//     the matching up outputs (the weight transform interleaves them);
+//     a = silu(gate) * up in FP32, requantised per 32 values to E4M3 + UE8M0
+//     ("DeepSeek DeepGEMM 2026年4月重磅更新" section 3.1: SwiGLU between
+//     linear1 and linear2; section 4.2: UE8M0 scale factors, four per int32).
+//   linear2 (kEpi 2): rows scaled by their top-k weight, written as FP32
+//     through swizzled shared-memory staging and TMA tensor stores.
+#pragma once
+
+#include "moe_device.cuh"
+#include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+
+constexpr int kEpiOutStage = 2048;  // bytes of staging per epilogue warp (32 rows x 16 FP32)
+
+// TMEM -> registers: the columns this thread's half of the epilogue needs.
+template <int kEpi>
+__device__ __forceinline__ void epilogue_load(uint32_t (&v)[4][32], uint32_t trow, int h) {
+  using namespace ptx;
+  if (kEpi == 1) {
+    tmem_ld_32x32b_x32(trow + 64 * h, v[0]);
+    tmem_ld_32x32b_x32(trow + 64 * h + 32, v[1]);
+    tmem_ld_32x32b_x32(trow + 128 + 64 * h, v[2]);
+    tmem_ld_32x32b_x32(trow + 128 + 64 * h + 32, v[3]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(trow + 128 * h + 32 * c, v[c]);
+  }
+}
+
+// Compute and store one (row, half) of a finished tile.  mt: m-tile (128
+// padded rows), nt: n-tile (256 weight rows), r: row in the tile, q: the
+// warp's 32-row group, stg: the warp's staging buffer.  Warp-collective for
+// kEpi 2 (all lanes must call it together).
+template <int kEpi>
+__device__ __forceinline__ void epilogue_store(const uint32_t (&v)[4][32], const GemmArgs& args,
+                                               const CUtensorMap* tmOut, uint8_t* stg, int mt,
+                                               int nt, int r, int h, int q, int lane) {
+  using namespace ptx;
+  const int row = mt * kBlockM + r;
+  const int src = args.src_of[row];
+  if (kEpi == 1) {
+    if (src < 0) return;  // padding row
+    uint32_t sbytes = 0;
+    uint8_t* dst = args.a2 + (size_t)row * args.I + nt * 128 + 64 * h;
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      float a[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float g = __uint_as_float(v[b][i]);
+        const float u = __uint_as_float(v[2 + b][i]);
+        a[i] = g * __frcp_rn(1.0f + __expf(-g)) * u;  // silu(g) * u
+      }
+      uint32_t packed[8], sb;
+      requant32(a, packed, sb);
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * b);
+      d4[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      d4[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+      sbytes |= sb << (8 * b);
+    }
+    uint8_t* sfdst = args.a2_sf + ((size_t)mt * (args.I / 128) + nt) * kSfChunk + (r & 31) * 16 +
+                     (r >> 5) * 4 + 2 * h;
+    *reinterpret_cast<uint16_t*>(sfdst) = (uint16_t)sbytes;
+  } else {
+    // 8 chunks of 32 rows x 16 columns per warp; 64-byte swizzled staging
+    const int col0 = nt * kBlockN + 128 * h;
+    if (col0 >= args.n_rows) return;  // half tile at the end of N (warp-uniform)
+    const float w = src >= 0 ? args.topk_w[src] : 0.0f;
+    const uint32_t stg_row = smem_u32(stg) + (uint32_t)lane * 64u;
+    const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (lane == 0) bulk_wait_group_read0();  // staging free again
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i0 = (c * 16 + j * 4) & 31, vb = (c * 16 + j * 4) >> 5;
+        st_shared_v4(stg_row + 16u * ((uint32_t)j ^ swz), w * __uint_as_float(v[vb][i0]),
+                     w * __uint_as_float(v[vb][i0 + 1]), w * __uint_as_float(v[vb][i0 + 2]),
+                     w * __uint_as_float(v[vb][i0 + 3]));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmOut, stg, col0 + 16 * c, mt * kBlockM + q * 32);
+        bulk_commit_group();
+      }
+    }
+  }
+}
+
+}  // namespace moe

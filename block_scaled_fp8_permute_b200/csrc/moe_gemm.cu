@@ -25,8 +25,7 @@
 // belongs to one expert (rows are padded per expert to 128).
 #include <cuda_fp8.h>
 
-#include "moe_internal.cuh"
-#include "sm100_ptx.cuh"
+#include "moe_epilogue.cuh"
 
 namespace moe {
 
@@ -41,45 +40,9 @@ constexpr int kGemmThreads = 64 + 32 * kNumEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;    // FP32 accumulator, 256 columns
 constexpr uint32_t kSfCol = 256;   // scale buffers: buf b -> SFA at +16b (4 cols), SFB at +16b+4 (8)
-constexpr int kOutStage = 2048;      // per epilogue warp: 32 rows x 16 FP32, 64-byte swizzle
+constexpr int kOutStage = kEpiOutStage;
 constexpr size_t kGemmSmemBytes = 1024 + (size_t)kStages * (kSmemA + kSmemB + kSmemSFA + kSmemSFB) +
                                   (size_t)kNumEpiWarps * kOutStage + 256;
-
-// ------------------------------------------------------------- requantiser
-// Smallest e with 448 * 2^e >= amax, from the bits of amax (448 = 1.75 * 2^8):
-// amax = m * 2^x with m in [1,2) needs e = x - 8 when m <= 1.75, else x - 7.
-// amax == 0 gives 0; results are clamped to [-127, 127].
-__device__ __forceinline__ int e4m3_block_exponent(float amax) {
-  const uint32_t bits = __float_as_uint(amax);
-  const int biased = (int)((bits >> 23) & 0xFF);
-  if (amax == 0.0f) return 0;
-  if (biased == 0) return -127;
-  const int x = biased - 127;
-  int e = ((bits & 0x7FFFFFu) > 0x600000u) ? x - 7 : x - 8;
-  return e < -127 ? -127 : (e > 127 ? 127 : e);
-}
-
-// Requantise 32 floats: E4M3 codes (little-endian packed, 4 per word) and
-// the UE8M0 byte of the block.
-__device__ __forceinline__ void requant32(const float (&a)[32], uint32_t (&packed)[8],
-                                          uint32_t& sbyte) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(a[i]));
-  const int e = e4m3_block_exponent(amax);
-  const float inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const __nv_fp8x2_storage_t lo =
-        __nv_cvt_float2_to_fp8x2(make_float2(a[4 * i] * inv, a[4 * i + 1] * inv), __NV_SATFINITE,
-                                 __NV_E4M3);
-    const __nv_fp8x2_storage_t hi =
-        __nv_cvt_float2_to_fp8x2(make_float2(a[4 * i + 2] * inv, a[4 * i + 3] * inv),
-                                 __NV_SATFINITE, __NV_E4M3);
-    packed[i] = (uint32_t)lo | ((uint32_t)hi << 16);
-  }
-  sbyte = (uint32_t)(e + 127);
-}
 
 __global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int cols,
                                      uint8_t* __restrict__ codes, uint8_t* __restrict__ sbytes) {
@@ -97,11 +60,6 @@ __global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int 
     dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
     sbytes[b] = (uint8_t)sb;
   }
-}
-
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // -------------------------------------------------------------------- kernel
@@ -272,74 +230,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after();
       uint32_t v[4][32];
-      if (kEpi == 1) {
-        // gate columns [64h, 64h+64), up columns [128+64h, 128+64h+64)
-        tmem_ld_32x32b_x32(trow + 64 * h, v[0]);
-        tmem_ld_32x32b_x32(trow + 64 * h + 32, v[1]);
-        tmem_ld_32x32b_x32(trow + 128 + 64 * h, v[2]);
-        tmem_ld_32x32b_x32(trow + 128 + 64 * h + 32, v[3]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(trow + 128 * h + 32 * c, v[c]);
-      }
+      epilogue_load<kEpi>(v, trow, h);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
-
-      const int row = mt * kBlockM + r;
-      const int src = args.src_of[row];
-      if (kEpi == 1) {
-        if (src < 0) continue;  // padding row (the loop head reconverges the warp)
-        uint32_t sbytes = 0;
-        uint8_t* dst = args.a2 + (size_t)row * args.I + nt * 128 + 64 * h;
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          float a[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float g = __uint_as_float(v[b][i]);
-            const float u = __uint_as_float(v[2 + b][i]);
-            a[i] = g * __frcp_rn(1.0f + __expf(-g)) * u;  // silu(g) * u
-          }
-          uint32_t packed[8], sb;
-          requant32(a, packed, sb);
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * b);
-          d4[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          d4[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-          sbytes |= sb << (8 * b);
-        }
-        uint8_t* sfdst = args.a2_sf + ((size_t)mt * (args.I / 128) + nt) * kSfChunk +
-                         (r & 31) * 16 + (r >> 5) * 4 + 2 * h;
-        *reinterpret_cast<uint16_t*>(sfdst) = (uint16_t)sbytes;
-      } else {
-        // weighted FP32 rows, written through shared memory by TMA stores:
-        // 8 chunks of 32 rows x 16 columns per warp (64-byte swizzled staging)
-        const int col0 = nt * kBlockN + 128 * h;
-        if (col0 >= n_rows) continue;  // half tile at the end of N (warp-uniform)
-        const float w = src >= 0 ? args.topk_w[src] : 0.0f;
-        uint8_t* stg = sOut + ew * kOutStage;
-        const uint32_t stg_row = smem_u32(stg) + (uint32_t)lane * 64u;
-        const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          if (lane == 0) bulk_wait_group_read0();  // staging free again
-          __syncwarp();
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int i0 = (c * 16 + j * 4) & 31, vb = (c * 16 + j * 4) >> 5;
-            st_shared_v4(stg_row + 16u * ((uint32_t)j ^ swz), w * __uint_as_float(v[vb][i0]),
-                         w * __uint_as_float(v[vb][i0 + 1]), w * __uint_as_float(v[vb][i0 + 2]),
-                         w * __uint_as_float(v[vb][i0 + 3]));
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmOut, stg, col0 + 16 * c, mt * kBlockM + q * 32);
-            bulk_commit_group();
-          }
-        }
-      }
+      epilogue_store<kEpi>(v, args, &tmOut, sOut + ew * kOutStage, mt, nt, r, h, q, lane);
     }
     if (kEpi == 2 && lane == 0) bulk_wait_group0();  // stores complete before the CTA exits
   }

@@ -26,15 +26,16 @@ enum HdrWord : int {
   kHdrMTiles = 2,     // P / kBlockM
   kHdrBadIds = 3,     // number of skipped invalid expert ids
   kHdrTimeoutSite = 4,
+  kHdrMPairs = 5,     // number of m-tile pairs (2-SM work rows)
   kHdrWords = 64
 };
 
 // byte offsets of every region of the workspace (all 1024-byte aligned)
 struct WsLayout {
-  size_t hdr, counts, offs, poffs, chunk, row_of, src_of, tile_expert;
+  size_t hdr, counts, offs, poffs, chunk, row_of, src_of, tile_expert, mpair;
   size_t xp, xp_sf, a2, a2_sf, yp;
   size_t total;
-  int R, P_max, MT_max, NCH;
+  int R, P_max, MT_max, MP_max, NCH;
 };
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -53,6 +54,8 @@ inline WsLayout ws_layout(const moe_shape& s) {
   L.R = s.T * s.topk;
   L.P_max = max_padded_rows(L.R, s.E);
   L.MT_max = L.P_max / kBlockM;
+  // pairs of m-tiles of one expert: at most one odd m-tile per non-empty expert
+  L.MP_max = L.MT_max / 2 + (L.R < s.E ? L.R : s.E) + 1;
   L.NCH = (L.R + kPlanChunk - 1) / kPlanChunk;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -68,6 +71,7 @@ inline WsLayout ws_layout(const moe_shape& s) {
   L.row_of = take((size_t)L.R * 4);
   L.src_of = take((size_t)L.P_max * 4);
   L.tile_expert = take((size_t)L.MT_max * 4);
+  L.mpair = take((size_t)L.MP_max * 4);
   L.xp = take((size_t)L.P_max * s.H);
   L.xp_sf = take((size_t)L.MT_max * (s.H / 128) * kSfChunk);
   L.a2 = take((size_t)L.P_max * s.I);
@@ -93,6 +97,7 @@ struct GemmArgs {
   float* yp;               // linear2 out: FP32 [P, H]
   const float* topk_w;     // [T*k]
   int H;
+  const int* mpair;        // m-tile pairs: first m-tile | (1 << 31) when the pair has one m-tile
 };
 
 // record the first error of a call in the status word

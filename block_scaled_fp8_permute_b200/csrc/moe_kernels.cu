@@ -48,18 +48,21 @@ __global__ void plan_count_kernel(const int32_t* __restrict__ idx, int R, int E,
 
 // K1b (one block of 1024 threads): turn chunk histograms into per-chunk
 // starting ranks (exclusive, in place), expert counts, offsets, padded
-// offsets, the m-tile -> expert table and -1 for padding rows of src_of.
+// offsets, the m-tile -> expert table, the list of m-tile pairs of one
+// expert (the work rows of the 2-SM GEMMs) and -1 for padding rows of src_of.
 __global__ void __launch_bounds__(1024) plan_scan_kernel(int E, int NCH, int* __restrict__ chunk_counts,
                                                          int* __restrict__ counts,
                                                          int* __restrict__ offs,
                                                          int* __restrict__ poffs,
                                                          int* __restrict__ tile_expert,
+                                                         int* __restrict__ mpair,
                                                          int* __restrict__ src_of,
                                                          int* __restrict__ hdr) {
-  __shared__ int warp_tot[2][32];
-  __shared__ int carry[2];
+  constexpr int NV = 3;  // scanned values: count, padded count, m-tile pairs
+  __shared__ int warp_tot[NV][32];
+  __shared__ int carry[NV];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  if (tid == 0) carry[0] = carry[1] = 0;
+  if (tid < NV) carry[tid] = 0;
   __syncthreads();
   for (int e0 = 0; e0 < E; e0 += 1024) {
     const int e = e0 + tid;
@@ -73,39 +76,48 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(int E, int NCH, int* __
       counts[e] = c;
     }
     const int pc = (c + kBlockM - 1) / kBlockM * kBlockM;
-    // block-wide inclusive scans of c and pc
-    int s0 = c, s1 = pc;
+    const int np = (pc / kBlockM + 1) / 2;
+    const int val[NV] = {c, pc, np};
+    int incl[NV] = {c, pc, np};
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-      const int t0 = __shfl_up_sync(0xffffffffu, s0, d), t1 = __shfl_up_sync(0xffffffffu, s1, d);
-      if (lane >= d) { s0 += t0; s1 += t1; }
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        const int t = __shfl_up_sync(0xffffffffu, incl[j], d);
+        if (lane >= d) incl[j] += t;
+      }
     }
-    if (lane == 31) { warp_tot[0][wid] = s0; warp_tot[1][wid] = s1; }
+    if (lane == 31)
+      for (int j = 0; j < NV; ++j) warp_tot[j][wid] = incl[j];
     __syncthreads();
     if (wid == 0) {
-      int w0 = warp_tot[0][lane], w1 = warp_tot[1][lane];
 #pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int t0 = __shfl_up_sync(0xffffffffu, w0, d), t1 = __shfl_up_sync(0xffffffffu, w1, d);
-        if (lane >= d) { w0 += t0; w1 += t1; }
+      for (int j = 0; j < NV; ++j) {
+        int w = warp_tot[j][lane];
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, w, d);
+          if (lane >= d) w += t;
+        }
+        warp_tot[j][lane] = w;
       }
-      warp_tot[0][lane] = w0;
-      warp_tot[1][lane] = w1;
     }
     __syncthreads();
-    const int pre0 = carry[0] + (wid ? warp_tot[0][wid - 1] : 0) + s0 - c;
-    const int pre1 = carry[1] + (wid ? warp_tot[1][wid - 1] : 0) + s1 - pc;
+    int pre[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+      pre[j] = carry[j] + (wid ? warp_tot[j][wid - 1] : 0) + incl[j] - val[j];
     if (e < E) {
-      offs[e] = pre0;
-      poffs[e] = pre1;
-      for (int mt = pre1 / kBlockM; mt < (pre1 + pc) / kBlockM; ++mt) tile_expert[mt] = e;
-      for (int r = pre1 + c; r < pre1 + pc; ++r) src_of[r] = -1;
+      offs[e] = pre[0];
+      poffs[e] = pre[1];
+      const int mt_first = pre[1] / kBlockM, nmt = pc / kBlockM;
+      for (int mt = mt_first; mt < mt_first + nmt; ++mt) tile_expert[mt] = e;
+      for (int i = 0; i < np; ++i)
+        mpair[pre[2] + i] = (mt_first + 2 * i) | ((2 * i + 1 == nmt) ? (int)0x80000000 : 0);
+      for (int r = pre[1] + c; r < pre[1] + pc; ++r) src_of[r] = -1;
     }
     __syncthreads();
-    if (tid == 0) {
-      carry[0] += warp_tot[0][31];
-      carry[1] += warp_tot[1][31];
-    }
+    if (tid < NV) carry[tid] += warp_tot[tid][31];
     __syncthreads();
   }
   if (tid == 0) {
@@ -113,6 +125,7 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(int E, int NCH, int* __
     poffs[E] = carry[1];
     hdr[kHdrP] = carry[1];
     hdr[kHdrMTiles] = carry[1] / kBlockM;
+    hdr[kHdrMPairs] = carry[2];
   }
 }
 
@@ -256,8 +269,8 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
 }
 
 cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int* chunk, int* counts,
-                        int* offs, int* poffs, int* tile_expert, int* row_of, int* src_of,
-                        int* hdr, cudaStream_t stream) {
+                        int* offs, int* poffs, int* tile_expert, int* mpair, int* row_of,
+                        int* src_of, int* hdr, cudaStream_t stream) {
   static bool attr_set = false;
   const size_t scatter_smem = (size_t)32 * E * sizeof(unsigned short);
   if (!attr_set) {
@@ -270,8 +283,8 @@ cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int* chunk, i
   if (R > 0) {
     plan_count_kernel<<<NCH, 256, E * sizeof(int), stream>>>(idx, R, E, chunk, hdr);
   }
-  plan_scan_kernel<<<1, 1024, 0, stream>>>(E, NCH, chunk, counts, offs, poffs, tile_expert, src_of,
-                                           hdr);
+  plan_scan_kernel<<<1, 1024, 0, stream>>>(E, NCH, chunk, counts, offs, poffs, tile_expert, mpair,
+                                           src_of, hdr);
   if (R > 0) {
     plan_scatter_kernel<<<NCH, 1024, scatter_smem, stream>>>(idx, R, E, chunk, poffs, row_of,
                                                              src_of);

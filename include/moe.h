@@ -97,6 +97,12 @@ void moe_set_num_sms(int num_sms);
  * (PDL moves kernel-to-kernel dependencies onto the GPU).  Default 1. */
 void moe_set_pdl(int enable);
 
+/* Tiling of the two grouped GEMMs: 0 (default) = one SM per 128 x 256
+ * output tile; 1 = SM pairs (thread-block clusters of 2, tcgen05
+ * cta_group::2) per 256 x 256 tile, used where the weight row count is a
+ * multiple of 256.  Both give identical results.  Process-wide. */
+void moe_set_gemm_variant(int variant);
+
 /* ---------------------------------------------------------------- weights */
 /* Bytes of one transformed weight: which = 1 for W1, 2 for W2.  Returns the
  * FP4 byte count and writes the scale-factor byte count to *sf_bytes (may

@@ -42,8 +42,16 @@ def _check_full(inputs, label):
     return lay, p
 
 
-def test_tiny_workload_all_tokens():
+def test_tiny_workload_all_tokens(gemm_variant):
     _check_full(synth.make_inputs(synth.workload("tiny")), "tiny")
+
+
+@pytest.fixture(params=[0, 1], ids=["one-sm", "sm-pair"])
+def gemm_variant(request):
+    import block_scaled_fp8_permute_b200 as moe
+    moe.moe_set_gemm_variant(request.param)
+    yield request.param
+    moe.moe_set_gemm_variant(0)
 
 
 @pytest.mark.parametrize("T,H,I,E,k", [
@@ -53,11 +61,11 @@ def test_tiny_workload_all_tokens():
     (130, 256, 384, 3, 3),     # m-tile tail: 130*3 rows over 3 experts
     (200, 512, 128, 64, 6),    # many experts, some empty
 ])
-def test_ragged_shapes_all_tokens(T, H, I, E, k):
+def test_ragged_shapes_all_tokens(T, H, I, E, k, gemm_variant):
     _check_full(_inputs(T, H, I, E, k, seed=T + H), f"T{T}H{H}I{I}E{E}k{k}")
 
 
-def test_unused_slots_duplicates_and_bad_ids():
+def test_unused_slots_duplicates_and_bad_ids(gemm_variant):
     d = _inputs(96, 256, 256, 6, 4, seed=5)
     idx = d["topk_idx"].copy()
     idx[::7, 1] = -1                 # unused slots
@@ -125,7 +133,7 @@ def _full_inputs(wl):
     ("mid", 96), ("usage", 12), ("skewed", 24), ("decode", 48), ("decode@T16", 16),
     ("decode@T32", 32), ("decode@T64", 32),
 ])
-def test_full_size_sampled(name, n_sample):
+def test_full_size_sampled(name, n_sample, gemm_variant):
     """Full-size workloads in the launch configuration bench.py uses; the
     oracle computes a seeded sample of tokens (first, last, random)."""
     wl = synth.workload(name)
