@@ -62,6 +62,7 @@ _SIGS = {
     "moe_plan_export": (_i, [_shp, _vp] + [_vp] * 6 + [_vp]),
     "moe_debug_requant": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "moe_set_timing_events": (None, [ctypes.POINTER(_vp), _i]),
+    "moe_forward_noalloc": (_i, [_shp] + [_vp] * 9 + [_vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -171,6 +172,15 @@ def moe_forward_host(shp, x, x_sf, topk_idx, topk_w, w1_t, w1_sf_t, w2_t, w2_sf_
         ctypes.byref(shp), _ptr(x), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(w1_t),
         _ptr(w1_sf_t), _ptr(w2_t), _ptr(w2_sf_t), _ptr(y), _ptr(workspace), ws_bytes,
         _stream(stream)))
+
+
+def moe_forward_noalloc(shp, x, x_sf, topk_idx, topk_w, w1_t, w1_sf_t, w2_t, w2_sf_t, y,
+                        stream=None):
+    """moe_plan + moe_forward on the library's own fixed 32 MiB workspace
+    (for callers that cannot allocate device memory)."""
+    _check("moe_forward_noalloc", _lib.moe_forward_noalloc(
+        ctypes.byref(shp), _ptr(x), _ptr(x_sf), _ptr(topk_idx), _ptr(topk_w), _ptr(w1_t),
+        _ptr(w1_sf_t), _ptr(w2_t), _ptr(w2_sf_t), _ptr(y), _stream(stream)))
 
 
 def moe_get_device_status(workspace, stream=None) -> int:

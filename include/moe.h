@@ -173,6 +173,36 @@ moe_status moe_forward_host(const moe_shape* shape, const uint8_t* x_host,
                             const void* w2_t, const void* w2_sf_t, uint16_t* y_host,
                             void* workspace, size_t ws_bytes, moe_stream_t stream);
 
+/* ---------------------------------------------------- allocation-free call */
+/* The pages describe no counterpart of this entry point; it exists for
+ * callers that cannot allocate device memory themselves: an inference
+ * runtime whose memory manager owns every device byte, code that runs while
+ * a CUDA graph is being captured, or a plug-in that is handed only its
+ * inputs and outputs.  It performs moe_plan + moe_forward with the
+ * workspace taken from a fixed 32 MiB array inside the library (a
+ * file-scope __device__ array: every GPU that loads the library holds those
+ * 32 MiB until the process exits).  The caller passes the inputs and y
+ * exactly as for moe_forward (device pointers, canonical layouts,
+ * transformed weights).
+ *   - Shapes whose moe_workspace_bytes() exceeds 32 MiB are rejected with
+ *     MOE_ERR_WORKSPACE before anything is launched (for example T = 256,
+ *     H = 2048, I = 1024, E = 8, top-2 fits; the large workloads do not).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Nothing is allocated: no cudaMalloc, no cudaFree, no allocating
+ *     library routine.  The header part of the array is cleared by every
+ *     call; the rest keeps the last call's contents and is rewritten before
+ *     it is read.
+ *   - All calls share the one array: calls whose GPU work overlaps (two
+ *     streams, two host threads) race and corrupt each other.  Order them
+ *     on one stream.
+ * Data-dependent problems (bad expert ids, device timeouts) are recorded in
+ * the array's status word as for moe_forward. */
+moe_status moe_forward_noalloc(const moe_shape* shape, const uint8_t* x, const int32_t* x_sf,
+                               const int32_t* topk_idx, const float* topk_w, const void* w1_t,
+                               const void* w1_sf_t, const void* w2_t, const void* w2_sf_t,
+                               uint16_t* y, moe_stream_t stream);
+
 /* ------------------------------------------------------------- diagnostics */
 /* Synchronises `stream` and returns the device status word of the last
  * plan / forward that used `workspace` (MOE_OK, MOE_ERR_BAD_EXPERT_ID or

@@ -1,0 +1,61 @@
+"""The allocation-free entry point, moe_forward_noalloc, for callers that
+cannot allocate device memory (a runtime whose allocator owns all device
+memory, code running under CUDA-graph capture, a plug-in handed only its
+inputs and outputs).  It must give what moe_forward gives, on two calls in a
+row (the second reuses the library's fixed workspace with its previous
+contents), and must reject shapes whose workspace exceeds its 32 MiB array.
+
+This file is collected last so that a run stopping at the first failure has
+already run every other test."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import synth
+from tests.gpu_util import Layer, assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _noalloc(lay, moe, idx=None):
+    import torch
+    d = lay.dev
+    y = torch.empty_like(lay.y)
+    moe.moe_forward_noalloc(lay.shape, d["x"], d["x_sf"], d["topk_idx"] if idx is None else idx,
+                            d["topk_w"], *lay.wt, y)
+    torch.cuda.synchronize()
+    T = lay.shape.T
+    return y[:T].view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def test_noalloc_matches_forward_on_two_calls():
+    import block_scaled_fp8_permute_b200 as moe
+    d = synth.make_inputs(synth.workload("tiny"))
+    lay = Layer(d).run()
+    y_ref = lay.y_bits()
+    y1 = _noalloc(lay, moe)
+    assert_parity(y1, y_ref, "noalloc call 1")
+    # a second call with a different routing, then the original again: the
+    # fixed workspace keeps the previous call's contents in between
+    import torch
+    idx2 = torch.flip(lay.dev["topk_idx"], dims=[1]).contiguous()
+    _noalloc(lay, moe, idx=idx2)
+    y2 = _noalloc(lay, moe)
+    assert_parity(y2, y_ref, "noalloc call 2")
+    assert np.array_equal(y1, y2)
+
+
+def test_noalloc_rejects_oversized_shapes():
+    import block_scaled_fp8_permute_b200 as moe
+    shp = moe.shape(4096, 2048, 1024, 32, 4)          # needs far more than 32 MiB
+    assert moe.moe_workspace_bytes(shp) > (32 << 20)
+    st = moe.lib().moe_forward_noalloc(ctypes.byref(shp), *([None] * 9), None)
+    assert st == 3                                      # MOE_ERR_WORKSPACE, nothing launched
