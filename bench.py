@@ -28,6 +28,26 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer fwd TFLOPS & tokens/s on 1 B200; % of tensor/HBM roofline"
+
+# DRAM traffic (read + write bytes) of one linear1 launch on the mid workload from an ncu
+# capture (profiles/gemm_mid.md).  Reported only while the kernel sources still hash to
+# the value they had when the counters were taken; otherwise the traffic is unknown (null).
+LINEAR1_TRAFFIC = {"workload": "mid", "bytes": 110.160896e6 + 8.945152e6,
+                   "sources_sha256_16": "1e20b863da6d3b8a"}
+LINEAR1_SOURCES = ["moe_gemm.cu", "moe_epilogue.cuh", "moe_device.cuh", "sm100_ptx.cuh",
+                   "moe_internal.cuh"]
+
+
+def _linear1_traffic(workload_name):
+    import hashlib
+    h = hashlib.sha256()
+    for f in LINEAR1_SOURCES:
+        with open(os.path.join(ROOT, "block_scaled_fp8_permute_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if (workload_name == LINEAR1_TRAFFIC["workload"]
+            and h.hexdigest()[:16] == LINEAR1_TRAFFIC["sources_sha256_16"]):
+        return LINEAR1_TRAFFIC["bytes"]
+    return None
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -315,7 +335,8 @@ def run_ours(args, wl, dist, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": "linear1 (moe_gemm_kernel<1>)",
                      "achieved": g1_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
-                     "frac": g1_tflops / tensor_peak, "traffic": None,
+                     "frac": g1_tflops / tensor_peak, "traffic": _linear1_traffic(wl.name),
+                     "traffic_unit": "bytes per launch (ncu dram read+write)",
                      "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"},
         "kernels_ms": kern,
         "step_roofline_frac": (wl.flops / (ms * 1e-3) / 1e12) / tensor_peak,
