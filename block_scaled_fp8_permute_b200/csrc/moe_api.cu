@@ -17,9 +17,12 @@ cudaError_t launch_gemm_pair(int epi, const CUtensorMap& tmA, const CUtensorMap&
                              bool pdl, cudaStream_t stream);
 cudaError_t launch_requant_debug(const float* a, int rows, int cols, uint8_t* codes,
                                  uint8_t* sbytes, cudaStream_t stream);
-cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int* chunk, int* counts,
-                        int* offs, int* poffs, int* tile_expert, int* mpair, int* row_of,
-                        int* src_of, int* hdr, cudaStream_t stream);
+cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max, int* chunk,
+                        int* counts, int* offs, int* poffs, int* tile_expert, int* mpair,
+                        int* norm_mtiles, int* swap_experts, int* row_of, int* src_of, int* hdr,
+                        bool pdl, cudaStream_t stream);
+cudaError_t launch_gemm_swap(int epi, const CUtensorMap& tmW, const CUtensorMap& tmX,
+                             const GemmArgs& args, int grid, bool pdl, cudaStream_t stream);
 cudaError_t launch_permute(const uint8_t* x, const int32_t* x_sf, const int* src_of,
                            const int* hdr, int H, int topk, uint8_t* xp, uint8_t* xp_sf, int grid,
                            bool pdl, cudaStream_t stream);
@@ -33,6 +36,7 @@ namespace {
 std::atomic<int> g_num_sms_cap{0};
 std::atomic<int> g_pdl{1};
 std::atomic<int> g_gemm_variant{0};
+std::atomic<int> g_swap_max{0};
 std::mutex g_ev_mu;
 cudaEvent_t g_events[5];
 bool g_events_on = false;
@@ -82,13 +86,13 @@ moe_status check_shape(const moe_shape* s) {
   return MOE_OK;
 }
 
-// activations [rows, K] uint8 E4M3: box 128 x 128, 128-byte swizzle
-bool encode_act(CUtensorMap* m, const void* base, int rows, int K) {
+// activations [rows, K] uint8 E4M3: box 128 x box_rows, 128-byte swizzle
+bool encode_act(CUtensorMap* m, const void* base, int rows, int K, int box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)K};
-  cuuint32_t box[2] = {128, 128};
+  cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -148,6 +152,8 @@ struct Ws {
   int* src_of() const { return reinterpret_cast<int*>(base + L.src_of); }
   int* tile_expert() const { return reinterpret_cast<int*>(base + L.tile_expert); }
   int* mpair() const { return reinterpret_cast<int*>(base + L.mpair); }
+  int* norm_mt() const { return reinterpret_cast<int*>(base + L.norm_mt); }
+  int* swap_e() const { return reinterpret_cast<int*>(base + L.swap_e); }
   uint8_t* xp() const { return base + L.xp; }
   uint8_t* xp_sf() const { return base + L.xp_sf; }
   uint8_t* a2() const { return base + L.a2; }
@@ -205,6 +211,10 @@ void moe_set_num_sms(int num_sms) { g_num_sms_cap.store(num_sms > 0 ? num_sms : 
 void moe_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
 
 void moe_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }
+
+void moe_set_swap_max(int rows) {
+  g_swap_max.store(rows < 0 ? 0 : (rows > kMaxSwapRows ? kMaxSwapRows : rows));
+}
 
 void moe_set_timing_events(void* const* events, int n) {
   std::lock_guard<std::mutex> lk(g_ev_mu);
@@ -265,9 +275,10 @@ moe_status moe_plan(const moe_shape* shape, const int32_t* topk_idx, void* works
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(ws.hdr(), 0, kHdrWords * 4, s);
   if (e == cudaSuccess)
-    e = launch_plan(topk_idx, ws.L.R, shape->E, ws.L.NCH, ws.chunk(), ws.counts(), ws.offs(),
-                    ws.poffs(), ws.tile_expert(), ws.mpair(), ws.row_of(), ws.src_of(), ws.hdr(),
-                    s);
+    e = launch_plan(topk_idx, ws.L.R, shape->E, ws.L.NCH, g_swap_max.load(), ws.chunk(),
+                    ws.counts(), ws.offs(), ws.poffs(), ws.tile_expert(), ws.mpair(),
+                    ws.norm_mt(), ws.swap_e(), ws.row_of(), ws.src_of(), ws.hdr(),
+                    g_pdl.load() != 0, s);
   return cuda_status(e);
 }
 
@@ -302,6 +313,12 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   const bool pair1 = g_gemm_variant.load() == 1;
   const bool pair2 = pair1 && (sh.H % 256) == 0;
   CUtensorMap tmX, tmW1, tmA2, tmW2, tmYp, tmXsf, tmW1sf, tmA2sf, tmW2sf;
+  CUtensorMap tmX16, tmA216, tmW1s, tmW2s;  // swapped-role kernel: 16-row token boxes
+  if (!encode_act(&tmX16, ws.xp(), ws.L.P_max, sh.H, 16) ||
+      !encode_act(&tmA216, ws.a2(), ws.L.P_max, sh.I, 16) ||
+      !encode_wgt(&tmW1s, w1_t, sh.E, KB1, 2 * sh.I, 256) ||
+      !encode_wgt(&tmW2s, w2_t, sh.E, KB2, sh.H, 256))
+    return MOE_ERR_CUDA;
   if (!encode_act(&tmX, ws.xp(), ws.L.P_max, sh.H) ||
       !encode_wgt(&tmW1, w1_t, sh.E, KB1, 2 * sh.I, pair1 ? 128 : 256) ||
       !encode_act(&tmA2, ws.a2(), ws.L.P_max, sh.I) ||
@@ -319,7 +336,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   if (pgrid > sms * 16) pgrid = sms * 16;
   if (pgrid < 1) pgrid = 1;
   cudaError_t e = launch_permute(x, x_sf, ws.src_of(), ws.hdr(), sh.H, sh.topk, ws.xp(),
-                                 ws.xp_sf(), pgrid, false, s);
+                                 ws.xp_sf(), pgrid, pdl, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   record_event(1, s);
 
@@ -331,6 +348,10 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   g1.tile_expert = ws.tile_expert();
   g1.src_of = ws.src_of();
   g1.mpair = ws.mpair();
+  g1.norm_mtiles = ws.norm_mt();
+  g1.swap_experts = ws.swap_e();
+  g1.poffs = ws.poffs();
+  g1.counts = ws.counts();
   g1.KB = KB1;
   g1.n_rows = 2 * sh.I;
   g1.NT = NT1;
@@ -347,6 +368,9 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
     int grid1 = (int)(tiles1 < sms ? tiles1 : sms);
     e = launch_gemm(1, tmX, tmW1, tmYp, g1, grid1 < 1 ? 1 : grid1, pdl, s);
   }
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const int swap_grid1 = (int)((long long)sh.E * NT1 < sms ? (long long)sh.E * NT1 : sms);
+  e = launch_gemm_swap(1, tmW1s, tmX16, g1, swap_grid1, pdl, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   record_event(2, s);
 
@@ -367,6 +391,9 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
     int grid2 = (int)(tiles2 < sms ? tiles2 : sms);
     e = launch_gemm(2, tmA2, tmW2, tmYp, g2, grid2 < 1 ? 1 : grid2, pdl, s);
   }
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const int swap_grid2 = (int)((long long)sh.E * NT2 < sms ? (long long)sh.E * NT2 : sms);
+  e = launch_gemm_swap(2, tmW2s, tmA216, g2, swap_grid2, pdl, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   record_event(3, s);
 

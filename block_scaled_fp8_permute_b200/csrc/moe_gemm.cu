@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   pdl_wait();  // inputs come from the previous kernel of the forward
   const int NT = args.NT, KB = args.KB, n_rows = args.n_rows;
-  const int num_tiles = args.hdr[kHdrMTiles] * NT;
+  const int num_tiles = args.hdr[kHdrNormMTiles] * NT;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t issued_mask = 0, last_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int mt = tile / NT, nt = tile - (tile / NT) * NT;
+        const int mt = args.norm_mtiles[tile / NT], nt = tile - (tile / NT) * NT;
         const int e = args.tile_expert[mt];
         const int n0 = nt * kBlockN;
         const uint32_t sfb_bytes = (n_rows - n0 > 128) ? 2 * kSfChunk : kSfChunk;
@@ -217,7 +217,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + kAccCol;
     int ti = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++ti) {
-      const int mt = tile / NT, nt = tile - (tile / NT) * NT;
+      const int mt = args.norm_mtiles[tile / NT], nt = tile - (tile / NT) * NT;
       // warp-uniform decision: every lane leaves or every lane continues
       const bool ready = __all_sync(0xffffffffu, mbar_wait(acc_full, ti & 1) && !*abort_flag);
       if (!ready) {

@@ -24,61 +24,83 @@ __device__ __forceinline__ size_t sf_chunk_offset(int row, int kg, int G) {
 }
 
 // ------------------------------------------------------------------- plan
-// K1a: per-chunk expert histograms.  chunk_counts[b][e] = assignments of
-// chunk b (kPlanChunk consecutive flattened slots) routed to expert e.
-__global__ void plan_count_kernel(const int32_t* __restrict__ idx, int R, int E,
-                                  int* __restrict__ chunk_counts, int* __restrict__ hdr) {
-  extern __shared__ int hist[];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+// K1 (count + scan, one launch): every block histograms its chunk of
+// kPlanChunk consecutive flattened slots into chunk_counts[b][e]; the last
+// block to finish then turns the chunk histograms into per-chunk starting
+// ranks (exclusive, in place), expert counts, offsets, padded offsets, the
+// m-tile -> expert table, the m-tile pairs and m-tiles of normal-tiled
+// experts, the list of swapped-role experts (1 <= count <= swap_max) and -1
+// for the padding rows of src_of.
+__global__ void __launch_bounds__(1024) plan_count_scan_kernel(
+    const int32_t* __restrict__ idx, int R, int E, int NCH, int swap_max,
+    int* __restrict__ chunk_counts, int* __restrict__ counts, int* __restrict__ offs,
+    int* __restrict__ poffs, int* __restrict__ tile_expert, int* __restrict__ mpair,
+    int* __restrict__ norm_mtiles, int* __restrict__ swap_experts, int* __restrict__ src_of,
+    int* __restrict__ hdr) {
+  __shared__ int hist[kMaxE];
+  __shared__ int last_block;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  const int base = blockIdx.x * kPlanChunk;
-  int bad = 0;
-  for (int i = threadIdx.x; i < kPlanChunk && base + i < R; i += blockDim.x) {
-    const int e = idx[base + i];
-    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
-    else if (e != -1) bad++;
-  }
-  if (bad) {
-    atomicAdd(&hdr[kHdrBadIds], bad);
-    set_status(hdr, MOE_ERR_BAD_EXPERT_ID);
+  const int a = blockIdx.x * kPlanChunk + tid;
+  if (a < R) {
+    const int e = idx[a];
+    if (e >= 0 && e < E) {
+      atomicAdd(&hist[e], 1);
+    } else if (e != -1) {
+      atomicAdd(&hdr[kHdrBadIds], 1);
+      set_status(hdr, MOE_ERR_BAD_EXPERT_ID);
+    }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[(size_t)blockIdx.x * E + e] = hist[e];
-}
+  if (R > 0)
+    for (int e = tid; e < E; e += blockDim.x) chunk_counts[(size_t)blockIdx.x * E + e] = hist[e];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last_block = atomicAdd(&hdr[kHdrPlanDone], 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!last_block) return;
+  __threadfence();
+  if (tid == 0) hdr[kHdrPlanDone] = 0;
 
-// K1b (one block of 1024 threads): turn chunk histograms into per-chunk
-// starting ranks (exclusive, in place), expert counts, offsets, padded
-// offsets, the m-tile -> expert table, the list of m-tile pairs of one
-// expert (the work rows of the 2-SM GEMMs) and -1 for padding rows of src_of.
-__global__ void __launch_bounds__(1024) plan_scan_kernel(int E, int NCH, int* __restrict__ chunk_counts,
-                                                         int* __restrict__ counts,
-                                                         int* __restrict__ offs,
-                                                         int* __restrict__ poffs,
-                                                         int* __restrict__ tile_expert,
-                                                         int* __restrict__ mpair,
-                                                         int* __restrict__ src_of,
-                                                         int* __restrict__ hdr) {
-  constexpr int NV = 3;  // scanned values: count, padded count, m-tile pairs
+  // ---- scan (last block only): count, padded count, m-tile pairs and
+  // m-tiles of the normal-tiled experts, swapped-role experts
+  constexpr int NV = 5;
   __shared__ int warp_tot[NV][32];
   __shared__ int carry[NV];
-  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  if (tid < NV) carry[tid] = 0;
+  const int lane = tid & 31, wid = tid >> 5;
+  if (tid < 5) carry[tid] = 0;
   __syncthreads();
   for (int e0 = 0; e0 < E; e0 += 1024) {
     const int e = e0 + tid;
     int c = 0;
-    if (e < E) {
-      for (int b = 0; b < NCH; ++b) {
+    if (e < E && R > 0) {
+      // chunk histograms of this expert: exclusive prefix in place, several loads in flight
+      int b = 0;
+      for (; b + 8 <= NCH; b += 8) {
+        int v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = chunk_counts[(size_t)(b + j) * E + e];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          chunk_counts[(size_t)(b + j) * E + e] = c;
+          c += v[j];
+        }
+      }
+      for (; b < NCH; ++b) {
         const int v = chunk_counts[(size_t)b * E + e];
         chunk_counts[(size_t)b * E + e] = c;
         c += v;
       }
-      counts[e] = c;
     }
+    if (e < E) counts[e] = c;
     const int pc = (c + kBlockM - 1) / kBlockM * kBlockM;
-    const int np = (pc / kBlockM + 1) / 2;
-    const int val[NV] = {c, pc, np};
-    int incl[NV] = {c, pc, np};
+    const bool swapped = c > 0 && c <= swap_max;
+    const int nm = swapped ? 0 : pc / kBlockM;
+    const int np = (nm + 1) / 2;
+    const int ns = swapped ? 1 : 0;
+    const int val[NV] = {c, pc, np, nm, ns};
+    int incl[NV] = {c, pc, np, nm, ns};
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
 #pragma unroll
@@ -113,7 +135,9 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(int E, int NCH, int* __
       const int mt_first = pre[1] / kBlockM, nmt = pc / kBlockM;
       for (int mt = mt_first; mt < mt_first + nmt; ++mt) tile_expert[mt] = e;
       for (int i = 0; i < np; ++i)
-        mpair[pre[2] + i] = (mt_first + 2 * i) | ((2 * i + 1 == nmt) ? (int)0x80000000 : 0);
+        mpair[pre[2] + i] = (mt_first + 2 * i) | ((2 * i + 1 == nm) ? (int)0x80000000 : 0);
+      for (int i = 0; i < nm; ++i) norm_mtiles[pre[3] + i] = mt_first + i;
+      if (swapped) swap_experts[pre[4]] = e;
       for (int r = pre[1] + c; r < pre[1] + pc; ++r) src_of[r] = -1;
     }
     __syncthreads();
@@ -126,10 +150,13 @@ __global__ void __launch_bounds__(1024) plan_scan_kernel(int E, int NCH, int* __
     hdr[kHdrP] = carry[1];
     hdr[kHdrMTiles] = carry[1] / kBlockM;
     hdr[kHdrMPairs] = carry[2];
+    hdr[kHdrNormMTiles] = carry[3];
+    hdr[kHdrSwapExperts] = carry[4];
+    hdr[kHdrSwapMax] = swap_max;
   }
 }
 
-// K1c: stable scatter.  Thread i of block b owns assignment b*kPlanChunk+i;
+// K2: stable scatter.  Thread i of block b owns assignment b*kPlanChunk+i;
 // its row is padded_offs[e] + (assignments of e in earlier chunks) +
 // (assignments of e in earlier warps of this chunk) + (earlier lanes of its
 // warp with the same expert), which orders each expert's rows by ascending
@@ -143,6 +170,7 @@ __global__ void __launch_bounds__(1024) plan_scatter_kernel(const int32_t* __res
   extern __shared__ unsigned short wcnt[];  // [32 warps][E]
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   for (int i = tid; i < 32 * E; i += blockDim.x) wcnt[i] = 0;
+  pdl_wait_k();  // chunk bases and padded offsets come from K1
   __syncthreads();
   const int a = blockIdx.x * kPlanChunk + tid;
   int e = -1;
@@ -268,9 +296,10 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int* chunk, int* counts,
-                        int* offs, int* poffs, int* tile_expert, int* mpair, int* row_of,
-                        int* src_of, int* hdr, cudaStream_t stream) {
+cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max, int* chunk,
+                        int* counts, int* offs, int* poffs, int* tile_expert, int* mpair,
+                        int* norm_mtiles, int* swap_experts, int* row_of, int* src_of, int* hdr,
+                        bool pdl, cudaStream_t stream) {
   static bool attr_set = false;
   const size_t scatter_smem = (size_t)32 * E * sizeof(unsigned short);
   if (!attr_set) {
@@ -280,16 +309,18 @@ cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int* chunk, i
     if (err != cudaSuccess) return err;
     attr_set = true;
   }
-  if (R > 0) {
-    plan_count_kernel<<<NCH, 256, E * sizeof(int), stream>>>(idx, R, E, chunk, hdr);
-  }
-  plan_scan_kernel<<<1, 1024, 0, stream>>>(E, NCH, chunk, counts, offs, poffs, tile_expert, mpair,
-                                           src_of, hdr);
-  if (R > 0) {
-    plan_scatter_kernel<<<NCH, 1024, scatter_smem, stream>>>(idx, R, E, chunk, poffs, row_of,
-                                                             src_of);
-  }
-  return cudaGetLastError();
+  plan_count_scan_kernel<<<NCH > 0 ? NCH : 1, 1024, 0, stream>>>(
+      idx, R, E, NCH, swap_max, chunk, counts, offs, poffs, tile_expert, mpair, norm_mtiles,
+      swap_experts, src_of, hdr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || R == 0) return e;
+  const int32_t* cidx = idx;
+  const int* cchunk = chunk;
+  const int* cpoffs = poffs;
+  void* args[] = {(void*)&cidx, (void*)&R, (void*)&E, (void*)&cchunk, (void*)&cpoffs,
+                  (void*)&row_of, (void*)&src_of};
+  return launch_pdl((const void*)plan_scatter_kernel, dim3(NCH), dim3(1024), scatter_smem, pdl,
+                    stream, args);
 }
 
 cudaError_t launch_permute(const uint8_t* x, const int32_t* x_sf, const int* src_of,

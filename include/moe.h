@@ -103,6 +103,14 @@ void moe_set_pdl(int enable);
  * multiple of 256.  Both give identical results.  Process-wide. */
 void moe_set_gemm_variant(int variant);
 
+/* Experts with at most `rows` routed rows (0..64; default 0 = off) run with
+ * swapped operand roles: the weights take the MMA's M side and the expert's
+ * rows the N side (N = rows rounded up to 16), so a decode-sized expert no
+ * longer pays for a 128-row tile ("DeepSeek DeepGEMM 2026年4月重磅更新" section
+ * 8.1, Dynamic Swap A/B).  Read by moe_plan; 0 disables.  Results are the
+ * same either way.  Process-wide. */
+void moe_set_swap_max(int rows);
+
 /* ---------------------------------------------------------------- weights */
 /* Bytes of one transformed weight: which = 1 for W1, 2 for W2.  Returns the
  * FP4 byte count and writes the scale-factor byte count to *sf_bytes (may

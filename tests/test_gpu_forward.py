@@ -46,12 +46,18 @@ def test_tiny_workload_all_tokens(gemm_variant):
     _check_full(synth.make_inputs(synth.workload("tiny")), "tiny")
 
 
-@pytest.fixture(params=[0, 1], ids=["one-sm", "sm-pair"])
+@pytest.fixture(params=[(0, 64), (0, 0), (1, 64), (1, 0)],
+                ids=["one-sm+swap", "one-sm", "sm-pair+swap", "sm-pair"])
 def gemm_variant(request):
+    """Tiling of the normal GEMM tiles x the swapped-role threshold (0: every
+    expert uses normal tiles; 64: experts with <= 64 rows use swapped roles)."""
     import block_scaled_fp8_permute_b200 as moe
-    moe.moe_set_gemm_variant(request.param)
+    variant, swap_max = request.param
+    moe.moe_set_gemm_variant(variant)
+    moe.moe_set_swap_max(swap_max)
     yield request.param
     moe.moe_set_gemm_variant(0)
+    moe.moe_set_swap_max(0)
 
 
 @pytest.mark.parametrize("T,H,I,E,k", [
@@ -60,6 +66,8 @@ def gemm_variant(request):
     (300, 384, 256, 16, 4),    # H = 384: one full and one half tile along N
     (130, 256, 384, 3, 3),     # m-tile tail: 130*3 rows over 3 experts
     (200, 512, 128, 64, 6),    # many experts, some empty
+    (600, 384, 256, 40, 3),    # mixed: experts above and below the swap threshold
+    (90, 256, 256, 2, 1),      # 45-ish rows per expert: swapped tiles of N = 48
 ])
 def test_ragged_shapes_all_tokens(T, H, I, E, k, gemm_variant):
     _check_full(_inputs(T, H, I, E, k, seed=T + H), f"T{T}H{H}I{I}E{E}k{k}")
@@ -129,11 +137,22 @@ def _full_inputs(wl):
     return dict(x=x, x_sf=x_sf, topk_idx=idx, topk_w=tw, w1=w1, w1_sf=w1_sf, w2=w2, w2_sf=w2_sf)
 
 
+@pytest.fixture(params=[(0, 0), (0, 64), (1, 0)], ids=["default", "swap", "sm-pair"])
+def full_variant(request):
+    import block_scaled_fp8_permute_b200 as moe
+    variant, swap_max = request.param
+    moe.moe_set_gemm_variant(variant)
+    moe.moe_set_swap_max(swap_max)
+    yield request.param
+    moe.moe_set_gemm_variant(0)
+    moe.moe_set_swap_max(0)
+
+
 @pytest.mark.parametrize("name,n_sample", [
     ("mid", 96), ("usage", 12), ("skewed", 24), ("decode", 48), ("decode@T16", 16),
     ("decode@T32", 32), ("decode@T64", 32),
 ])
-def test_full_size_sampled(name, n_sample, gemm_variant):
+def test_full_size_sampled(name, n_sample, full_variant):
     """Full-size workloads in the launch configuration bench.py uses; the
     oracle computes a seeded sample of tokens (first, last, random)."""
     wl = synth.workload(name)
