@@ -369,9 +369,13 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
     e = launch_gemm(1, tmX, tmW1, tmYp, g1, grid1 < 1 ? 1 : grid1, pdl, s);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  const int swap_grid1 = (int)((long long)sh.E * NT1 < sms ? (long long)sh.E * NT1 : sms);
-  e = launch_gemm_swap(1, tmW1s, tmX16, g1, swap_grid1, pdl, s);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  // swapped-role tiles exist only when the plan was made with a threshold > 0
+  const bool use_swap = g_swap_max.load() > 0;
+  if (use_swap) {
+    const int swap_grid1 = (int)((long long)sh.E * NT1 < sms ? (long long)sh.E * NT1 : sms);
+    e = launch_gemm_swap(1, tmW1s, tmX16, g1, swap_grid1, pdl, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
   record_event(2, s);
 
   GemmArgs g2 = g1;
@@ -392,9 +396,11 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
     e = launch_gemm(2, tmA2, tmW2, tmYp, g2, grid2 < 1 ? 1 : grid2, pdl, s);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  const int swap_grid2 = (int)((long long)sh.E * NT2 < sms ? (long long)sh.E * NT2 : sms);
-  e = launch_gemm_swap(2, tmW2s, tmA216, g2, swap_grid2, pdl, s);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (use_swap) {
+    const int swap_grid2 = (int)((long long)sh.E * NT2 < sms ? (long long)sh.E * NT2 : sms);
+    e = launch_gemm_swap(2, tmW2s, tmA216, g2, swap_grid2, pdl, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
   record_event(3, s);
 
   int cgrid = sh.T < 65535 ? sh.T : 65535;

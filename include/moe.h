@@ -107,8 +107,9 @@ void moe_set_gemm_variant(int variant);
  * swapped operand roles: the weights take the MMA's M side and the expert's
  * rows the N side (N = rows rounded up to 16), so a decode-sized expert no
  * longer pays for a 128-row tile ("DeepSeek DeepGEMM 2026年4月重磅更新" section
- * 8.1, Dynamic Swap A/B).  Read by moe_plan; 0 disables.  Results are the
- * same either way.  Process-wide. */
+ * 8.1, Dynamic Swap A/B).  Read by moe_plan and moe_forward, which must see
+ * the same value (set it before moe_plan); 0 disables.  Results are the same
+ * either way.  Process-wide. */
 void moe_set_swap_max(int rows);
 
 /* ---------------------------------------------------------------- weights */
