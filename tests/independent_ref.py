@@ -92,8 +92,21 @@ def bf16_round(v: np.ndarray) -> np.ndarray:
     return t.view(torch.int16).numpy().view(np.uint16)
 
 
+def bf16_value(v: np.ndarray) -> np.ndarray:
+    """float64 -> nearest bf16 value (ties to even), returned as float64.
+
+    bf16 keeps 8 significant bits: with |v| = m * 2^e, m in [0.5, 1), the
+    grid step is 2^(e-8); below 2^-126 the step stays 2^-133 (subnormals)."""
+    v = np.asarray(v, np.float64)
+    _, e = np.frexp(np.abs(v))
+    e = np.maximum(e, -125)
+    q = np.ldexp(np.rint(np.ldexp(np.abs(v), 8 - e)), e - 8)
+    return np.copysign(q, v)
+
+
 def moe_masked(x, x_sf, topk_idx, topk_w, w1, w1_sf, w2, w2_sf):
-    """Masked all-experts formulation: acc[t] = sum_e sum_s [idx[t,s]==e] w[t,s] FFN_e(x_t).
+    """Masked all-experts formulation:
+    acc[t] = sum_e sum_s [idx[t,s]==e] bf16(w[t,s] FFN_e(x_t)).
 
     Returns the float64 accumulator [T, H]."""
     T, H = x.shape
@@ -111,5 +124,5 @@ def moe_masked(x, x_sf, topk_idx, topk_w, w1, w1_sf, w2, w2_sf):
         O = ad @ W2[e].T                                  # [T, H]
         for s in range(topk_idx.shape[1]):
             sel = (topk_idx[:, s] == e).astype(np.float64) * topk_w[:, s].astype(np.float64)
-            acc += sel[:, None] * O
+            acc += bf16_value(sel[:, None] * O)
     return acc

@@ -147,6 +147,25 @@ def test_bf16_matches_torch_cast():
     assert np.array_equal(got, want)
 
 
+def test_bf16_of_doubles_matches_independent_rounding():
+    """Doubles that are not float32 values (the linear2 products the oracle
+    rounds): the oracle's rounding against the numpy formulation in
+    independent_ref, including exact ties and values a hair off a tie."""
+    import independent_ref as ind
+    rng = np.random.default_rng(7)
+    v = rng.standard_normal(3000) * np.exp2(rng.integers(-40, 40, 3000))
+    base = np.ldexp(rng.integers(128, 256, 500).astype(np.float64), rng.integers(-20, 20, 500))
+    ulp = np.ldexp(1.0, np.frexp(base)[1] - 8)
+    ties = base + 0.5 * ulp
+    v = np.concatenate([v, ties, -ties, ties + ulp * 1e-9, ties - ulp * 1e-9])
+    got = np.array([oracle.bf16_rne(float(a)) for a in v], np.uint16)
+    want = ind.bf16_value(v)
+    got_v = (got.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(got_v, want)
+    # exact ties go to the even neighbour: the significand's low bit is clear
+    assert ((got[3000:3500] & 1) == 0).all()
+
+
 def test_requant_block_matches_independent_formulation():
     from tests.independent_ref import requant
     rng = np.random.default_rng(2)

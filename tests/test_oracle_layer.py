@@ -141,7 +141,7 @@ def test_dense_ffn_special_case():
     G = X @ W1.T
     a = (G[:, :128] / (1 + np.exp(-G[:, :128])) * G[:, 128:]).astype(np.float32)
     ad, _, _ = ind.requant(a)
-    ref = ad @ W2.T
+    ref = ind.bf16_value(ad @ W2.T)  # the GEMM's BF16 output, weight 1
     np.testing.assert_allclose(acc, ref, rtol=1e-11, atol=1e-12 * np.abs(ref).max())
 
 
