@@ -26,8 +26,8 @@ cudaError_t launch_gemm_swap(int epi, const CUtensorMap& tmW, const CUtensorMap&
 cudaError_t launch_permute(const uint8_t* x, const int32_t* x_sf, const int* src_of,
                            const int* hdr, int H, int topk, uint8_t* xp, uint8_t* xp_sf, int grid,
                            bool pdl, cudaStream_t stream);
-cudaError_t launch_combine(const float* yp, const int* row_of, int T, int H, int topk, uint16_t* y,
-                           int grid, bool pdl, cudaStream_t stream);
+cudaError_t launch_combine(const uint16_t* yp, const int* row_of, int T, int H, int topk,
+                           uint16_t* y, int grid, bool pdl, cudaStream_t stream);
 cudaError_t launch_transform(const uint8_t* w, const uint8_t* w_sf, int E, int N, int K,
                              int interleave, uint8_t* wt, uint8_t* wt_sf, cudaStream_t stream);
 
@@ -113,15 +113,15 @@ bool encode_wgt(CUtensorMap* m, const void* base, int E, int KB, int n_rows, int
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// FP32 partial rows [rows, N]: TMA store box 16 columns x 32 rows, 64-byte swizzle
-bool encode_out_f32(CUtensorMap* m, const void* base, int rows, int N) {
+// BF16 partial rows [rows, N]: TMA store box 32 columns x 32 rows, 64-byte swizzle
+bool encode_out_bf16(CUtensorMap* m, const void* base, int rows, int N) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)N * 4};
-  cuuint32_t box[2] = {16, 32};
+  cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+  cuuint32_t box[2] = {32, 32};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -158,7 +158,7 @@ struct Ws {
   uint8_t* xp_sf() const { return base + L.xp_sf; }
   uint8_t* a2() const { return base + L.a2; }
   uint8_t* a2_sf() const { return base + L.a2_sf; }
-  float* yp() const { return reinterpret_cast<float*>(base + L.yp); }
+  uint16_t* yp() const { return reinterpret_cast<uint16_t*>(base + L.yp); }
 };
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -323,7 +323,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
       !encode_wgt(&tmW1, w1_t, sh.E, KB1, 2 * sh.I, pair1 ? 128 : 256) ||
       !encode_act(&tmA2, ws.a2(), ws.L.P_max, sh.I) ||
       !encode_wgt(&tmW2, w2_t, sh.E, KB2, sh.H, pair2 ? 128 : 256) ||
-      !encode_out_f32(&tmYp, ws.yp(), ws.L.P_max, sh.H) ||
+      !encode_out_bf16(&tmYp, ws.yp(), ws.L.P_max, sh.H) ||
       !encode_sf(&tmXsf, ws.xp_sf(), (long long)ws.L.MT_max * KB1, 1) ||
       !encode_sf(&tmW1sf, w1_sf_t, (long long)sh.E * KB1 * (2 * sh.I / 128), 2) ||
       !encode_sf(&tmA2sf, ws.a2_sf(), (long long)ws.L.MT_max * KB2, 1) ||

@@ -6,9 +6,12 @@
 //     a = silu(gate) * up in FP32, requantised per 32 values to E4M3 + UE8M0
 //     ("DeepSeek DeepGEMM 2026年4月重磅更新" section 3.1: SwiGLU between
 //     linear1 and linear2; section 4.2: UE8M0 scale factors, four per int32).
-//   linear2 (kEpi 2): rows scaled by their top-k weight, written as FP32
-//     through swizzled shared-memory staging and TMA tensor stores.
+//   linear2 (kEpi 2): rows scaled by their top-k weight, rounded to BF16
+//     (the GEMM's output type, section 4.3) and written through swizzled
+//     shared-memory staging and TMA tensor stores.
 #pragma once
+
+#include <cuda_bf16.h>
 
 #include "moe_device.cuh"
 #include "moe_internal.cuh"
@@ -16,7 +19,7 @@
 
 namespace moe {
 
-constexpr int kEpiOutStage = 2048;  // bytes of staging per epilogue warp (32 rows x 16 FP32)
+constexpr int kEpiOutStage = 2048;  // bytes of staging per epilogue warp (32 rows x 32 BF16)
 
 // TMEM -> registers: the columns this thread's half of the epilogue needs.
 template <int kEpi>
@@ -68,27 +71,31 @@ __device__ __forceinline__ void epilogue_store(const uint32_t (&v)[4][32], const
                      (r >> 5) * 4 + 2 * h;
     *reinterpret_cast<uint16_t*>(sfdst) = (uint16_t)sbytes;
   } else {
-    // 8 chunks of 32 rows x 16 columns per warp; 64-byte swizzled staging
+    // BF16 rows: 4 chunks of 32 rows x 32 columns per warp; 64-byte swizzled staging
     const int col0 = nt * kBlockN + 128 * h;
     if (col0 >= args.n_rows) return;  // half tile at the end of N (warp-uniform)
     const float w = src >= 0 ? args.topk_w[src] : 0.0f;
     const uint32_t stg_row = smem_u32(stg) + (uint32_t)lane * 64u;
     const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
       if (lane == 0) bulk_wait_group_read0();  // staging free again
       __syncwarp();
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int i0 = (c * 16 + j * 4) & 31, vb = (c * 16 + j * 4) >> 5;
-        st_shared_v4(stg_row + 16u * ((uint32_t)j ^ swz), w * __uint_as_float(v[vb][i0]),
-                     w * __uint_as_float(v[vb][i0 + 1]), w * __uint_as_float(v[vb][i0 + 2]),
-                     w * __uint_as_float(v[vb][i0 + 3]));
+        uint32_t p[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 b = __floats2bfloat162_rn(w * __uint_as_float(v[c][8 * j + 2 * i]),
+                                                         w * __uint_as_float(v[c][8 * j + 2 * i + 1]));
+          p[i] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        st_shared_v4(stg_row + 16u * ((uint32_t)j ^ swz), p[0], p[1], p[2], p[3]);
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_2d(tmOut, stg, col0 + 16 * c, mt * kBlockM + q * 32);
+        tma_store_2d(tmOut, stg, col0 + 32 * c, mt * kBlockM + q * 32);
         bulk_commit_group();
       }
     }

@@ -5,7 +5,7 @@
 //            UE8M0 scale per 1x32 block on both sides, FP32 accumulation) with
 //            the SwiGLU + E4M3 requantisation epilogue fused in;
 //   linear2: O = A2_e . W2_e^T with the top-k weight applied in the epilogue,
-//            FP32 partial rows written in expert-contiguous row order.
+//            BF16 partial rows written in expert-contiguous row order.
 // ("DeepSeek DeepGEMM 2026年4月重磅更新：Mega MoE融合算子、FP4精度与极致性能优化",
 //  section 3.2 (fusing linear1 / SwiGLU / linear2), section 4.2 (UE8M0 scale
 //  factors, FP32 accumulation), section 11.3 (TMA multi-stage loads).)
@@ -63,7 +63,7 @@ __global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int 
 }
 
 // -------------------------------------------------------------------- kernel
-template <int kEpi>  // 1: SwiGLU + requant (linear1), 2: x topk_w, FP32 rows (linear2)
+template <int kEpi>  // 1: SwiGLU + requant (linear1), 2: x topk_w, BF16 rows (linear2)
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,

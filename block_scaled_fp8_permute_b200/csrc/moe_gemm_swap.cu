@@ -13,7 +13,7 @@
 //            one output j for every token; the 32 outputs of a requant block
 //            are the 32 lanes of a warp (amax by warp reduction).
 //   linear2: MMA 0 / MMA 1 cover output columns h0..h0+127 / h0+128..h0+255;
-//            one warp writes 32 consecutive FP32 outputs of a token row.
+//            one warp writes 32 consecutive BF16 outputs of a token row.
 // Work item = (expert, 256-row weight group); each item streams that group's
 // weights once, so the kernel is bound by HBM weight traffic.
 //
@@ -276,9 +276,9 @@ __global__ void __launch_bounds__(swapk::kThreads, 1)
               const int row = r0 + t;
               const int src = args.src_of[row];
               const float w = args.topk_w[src];
-              float* dst = args.yp + (size_t)row * args.H;
-              dst[hc0] = w * __uint_as_float(g[i][c]);
-              if (hc0 + 128 < n_rows) dst[hc0 + 128] = w * __uint_as_float(u[i][c]);
+              __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(args.yp) + (size_t)row * args.H;
+              dst[hc0] = __float2bfloat16_rn(w * __uint_as_float(g[i][c]));
+              if (hc0 + 128 < n_rows) dst[hc0 + 128] = __float2bfloat16_rn(w * __uint_as_float(u[i][c]));
             }
           }
         }

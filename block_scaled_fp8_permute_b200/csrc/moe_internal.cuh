@@ -82,7 +82,7 @@ inline WsLayout ws_layout(const moe_shape& s) {
   L.xp_sf = take((size_t)L.MT_max * (s.H / 128) * kSfChunk);
   L.a2 = take((size_t)L.P_max * s.I);
   L.a2_sf = take((size_t)L.MT_max * (s.I / 128) * kSfChunk);
-  L.yp = take((size_t)L.P_max * s.H * 4);
+  L.yp = take((size_t)L.P_max * s.H * 2);
   L.total = off;
   return L;
 }
@@ -100,7 +100,7 @@ struct GemmArgs {
   uint8_t* a2;             // linear1 out: E4M3 [P, I]
   uint8_t* a2_sf;          // linear1 out: scale chunks [MT][I/128][512]
   int I;
-  float* yp;               // linear2 out: FP32 [P, H]
+  uint16_t* yp;            // linear2 out: BF16 [P, H], rows times their top-k weight
   const float* topk_w;     // [T*k]
   int H;
   const int* mpair;        // m-tile pairs: first m-tile | (1 << 31) when the pair has one m-tile

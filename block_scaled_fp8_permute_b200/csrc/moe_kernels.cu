@@ -2,7 +2,7 @@
 //   plan    (routing bookkeeping: histogram, prefix sums, stable scatter),
 //   permute (dispatch: gather token rows and their scales into
 //            expert-contiguous order),
-//   combine (weighted top-k reduction of the FP32 partial rows into BF16),
+//   combine (top-k reduction of the weighted BF16 partial rows into BF16),
 //   transform (one-time weight repack).
 // ("DeepSeek DeepGEMM 2026年4月重磅更新：Mega MoE融合算子、FP4精度与极致性能优化",
 //  section 3.1: the dispatch and combine steps around the two expert linears;
@@ -220,30 +220,40 @@ __global__ void permute_kernel(const uint8_t* __restrict__ x, const int32_t* __r
 }
 
 // ---------------------------------------------------------------- combine
-// y[t] = BF16_RNE( sum_s Yp[row_of[t][s]] ) in slot order, FP32 (the top-k
-// weight was applied by the linear2 epilogue).  One block per token.
-__global__ void combine_kernel(const float* __restrict__ yp, const int* __restrict__ row_of, int T,
-                               int H, int topk, __nv_bfloat16* __restrict__ y) {
+// y[t] = BF16_RNE( sum_s Yp[row_of[t][s]] ), slot order, FP32 sum of the
+// BF16 partial rows (the top-k weight was applied by the linear2 epilogue).
+// One block per token, 8 columns (16 bytes) per thread and slot.
+__global__ void combine_kernel(const uint16_t* __restrict__ yp, const int* __restrict__ row_of,
+                               int T, int H, int topk, __nv_bfloat16* __restrict__ y) {
   pdl_wait_k();
   __shared__ int rows[kMaxTopk];
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
     if (threadIdx.x < topk) rows[threadIdx.x] = row_of[(size_t)t * topk + threadIdx.x];
     __syncthreads();
-    for (int c = threadIdx.x * 4; c < H; c += blockDim.x * 4) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = threadIdx.x * 8; c < H; c += blockDim.x * 8) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll 4
       for (int s = 0; s < topk; ++s) {
         const int r = rows[s];
         if (r < 0) continue;
-        const float4 v = __ldg(reinterpret_cast<const float4*>(yp + (size_t)r * H + c));
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(yp + (size_t)r * H + c));
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] += __uint_as_float(w4[i] << 16);
+          acc[2 * i + 1] += __uint_as_float(w4[i] & 0xFFFF0000u);
+        }
       }
-      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-      uint2 packed;
-      packed.x = *reinterpret_cast<uint32_t*>(&lo);
-      packed.y = *reinterpret_cast<uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(y + (size_t)t * H + c) = packed;
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        o[i] = *reinterpret_cast<const uint32_t*>(&b);
+      }
+      *reinterpret_cast<uint4*>(y + (size_t)t * H + c) = make_uint4(o[0], o[1], o[2], o[3]);
     }
   }
   pdl_launch_k();
@@ -331,11 +341,11 @@ cudaError_t launch_permute(const uint8_t* x, const int32_t* x_sf, const int* src
   return launch_pdl((const void*)permute_kernel, dim3(grid), dim3(256), 0, pdl, stream, args);
 }
 
-cudaError_t launch_combine(const float* yp, const int* row_of, int T, int H, int topk, uint16_t* y,
-                           int grid, bool pdl, cudaStream_t stream) {
+cudaError_t launch_combine(const uint16_t* yp, const int* row_of, int T, int H, int topk,
+                           uint16_t* y, int grid, bool pdl, cudaStream_t stream) {
   __nv_bfloat16* yb = reinterpret_cast<__nv_bfloat16*>(y);
   void* args[] = {(void*)&yp, (void*)&row_of, (void*)&T, (void*)&H, (void*)&topk, (void*)&yb};
-  int threads = H / 4 < 256 ? ((H / 4 + 31) / 32) * 32 : 256;
+  int threads = H / 8 < 256 ? ((H / 8 + 31) / 32) * 32 : 256;
   return launch_pdl((const void*)combine_kernel, dim3(grid), dim3(threads), 0, pdl, stream, args);
 }
 

@@ -21,7 +21,8 @@
  *   a'  = E4M3 requantisation of a, one UE8M0 scale per 32 consecutive values,
  *         scale exponent = smallest e with 448 * 2^e >= amax (0 for amax 0)
  *   o   = W2[e] . a'                         (H outputs)
- *   y[t] = BF16_RNE( sum over s in slot order of topk_w[t][s] * o )   (FP32 sum)
+ *   p_s = BF16_RNE( topk_w[t][s] * o )       (the GEMM's BF16 output, section 4.3)
+ *   y[t] = BF16_RNE( sum over s in slot order of p_s )                 (FP32 sum)
  * All products are block-scaled: every 1x32 block along K of x, W1, W2 and a'
  * carries one UE8M0 scale (value 2^(b-127)).
  *
@@ -141,7 +142,7 @@ moe_status moe_transform_weights(const moe_shape* shape, const uint8_t* w1, cons
 /* -------------------------------------------------------------- workspace */
 /* Bytes of workspace one forward needs for this shape: the plan, the
  * permuted activations and their scales, the requantised intermediate and
- * its scales, and the FP32 weighted partial outputs.  It is an upper bound
+ * its scales, and the BF16 weighted partial outputs.  It is an upper bound
  * over every possible routing (rows padded per expert to moe_block_m()). */
 size_t moe_workspace_bytes(const moe_shape* shape);
 
