@@ -74,6 +74,8 @@ __device__ __forceinline__ void epilogue_store(const uint32_t (&v)[4][32], const
     // BF16 rows: 4 chunks of 32 rows x 32 columns per warp; 64-byte swizzled staging
     const int col0 = nt * kBlockN + 128 * h;
     if (col0 >= args.n_rows) return;  // half tile at the end of N (warp-uniform)
+    // 32 padding rows (an expert's last m-tile, decode-sized batches): nothing to store
+    if (__all_sync(0xffffffffu, src < 0)) return;
     const float w = src >= 0 ? args.topk_w[src] : 0.0f;
     const uint32_t stg_row = smem_u32(stg) + (uint32_t)lane * 64u;
     const uint32_t swz = ((uint32_t)lane >> 1) & 3u;
