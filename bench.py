@@ -29,11 +29,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer fwd TFLOPS & tokens/s on 1 B200; % of tensor/HBM roofline"
 
-# DRAM traffic (read + write bytes) of one linear1 launch on the mid workload from an ncu
-# capture (profiles/gemm_mid.md).  Reported only while the kernel sources still hash to
-# the value they had when the counters were taken; otherwise the traffic is unknown (null).
-LINEAR1_TRAFFIC = {"workload": "mid", "bytes": 110.160896e6 + 8.945152e6,
-                   "sources_sha256_16": "1e20b863da6d3b8a"}
+# DRAM traffic (read + write bytes) of one linear1 launch on the mid workload from one ncu
+# capture (summarised, with its command, under profiles/).  Reported only while the kernel
+# sources still hash to the value they had when the counters were taken; otherwise the
+# traffic is unknown (null).
+LINEAR1_TRAFFIC = {"workload": "mid", "bytes": 110.118656e6 + 8.988416e6,
+                   "sources_sha256_16": "9f557049bbf1796f"}
 LINEAR1_SOURCES = ["moe_gemm.cu", "moe_epilogue.cuh", "moe_device.cuh", "sm100_ptx.cuh",
                    "moe_internal.cuh"]
 
@@ -341,8 +342,30 @@ def run_ours(args, wl, dist, rank, world, local_rank):
     value = flops / (ms * 1e-3) / 1e12
     pk = _peaks()
     tensor_peak = 2.0 * pk["bf16"]  # FP8-rate MMA = 2 x the measured bf16 rate
-    g1_flops = 4.0 * wl.R * wl.H * wl.I
-    g1_tflops = g1_flops / (g1 * 1e-3) / 1e12
+    hbm_peak = pk["hbm"]
+    # Algorithmic bytes: the weights of the experts that receive rows (FP4 codes +
+    # one UE8M0 byte per 32) are read once; activations, intermediate and output once.
+    idx = inputs["topk_idx"]
+    R_valid = int((idx >= 0).sum())
+    touched = len(np.unique(idx[idx >= 0]))
+    H, I = wl.H, wl.I
+    w1_bytes = touched * (2 * I * H // 2 + 2 * I * H // 32)
+    w2_bytes = touched * (H * I // 2 + H * I // 32)
+    g1_flops = 4.0 * R_valid * H * I
+    g1_bytes = w1_bytes + R_valid * (H + H // 32) + R_valid * (I + I // 32)
+    step_bytes = (w1_bytes + w2_bytes + wl.T * (H + H // 32) + wl.T * wl.k * 8 + wl.T * H * 2)
+    # roofline time = the slower of the FLOPs at the tensor peak and the bytes at HBM bandwidth
+    g1_t_tensor = g1_flops / (tensor_peak * 1e12)
+    g1_t_hbm = g1_bytes / (hbm_peak * 1e9)
+    if g1_t_tensor >= g1_t_hbm:
+        roof = {"bound": "tensor", "achieved": g1_flops / (g1 * 1e-3) / 1e12, "peak": tensor_peak,
+                "unit": "TFLOP/s",
+                "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"}
+    else:
+        roof = {"bound": "hbm", "achieved": g1_bytes / (g1 * 1e-3) / 1e9, "peak": hbm_peak,
+                "unit": "GB/s", "peak_note": f"copy bandwidth {hbm_peak} GB/s ({pk['src']})"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    step_t_roof = max(wl.flops / (tensor_peak * 1e12), step_bytes / (hbm_peak * 1e9))
     cpu = None
     if not args.no_cpu_baseline:
         cv, n, sec, cores = _oracle_sample(wl, inputs, args.cpu_seconds)
@@ -358,14 +381,17 @@ def run_ours(args, wl, dist, rank, world, local_rank):
                    "l2": "flushed (256 MB write) before every timed step",
                    "step": "moe_plan + moe_forward replayed as one CUDA graph",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "tensor", "kernel": "linear1 (moe_gemm_kernel<1>)",
-                     "achieved": g1_tflops, "peak": tensor_peak, "unit": "TFLOP/s",
-                     "frac": g1_tflops / tensor_peak, "traffic": _linear1_traffic(wl.name),
-                     "traffic_unit": "bytes per launch (ncu dram read+write)",
-                     "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"},
+        "roofline": dict(roof, kernel="linear1 (moe_gemm_kernel<1>)",
+                         flops_per_launch=g1_flops, algorithmic_bytes_per_launch=g1_bytes,
+                         traffic=_linear1_traffic(wl.name),
+                         traffic_unit="bytes per launch (ncu dram read+write)"),
         "kernels_ms": kern,
         "kernels_ms_note": "eager steps with events at kernel boundaries (K extra steps)",
-        "step_roofline_frac": (wl.flops / (ms * 1e-3) / 1e12) / tensor_peak,
+        "step_roofline": {"bound": ("tensor" if wl.flops / (tensor_peak * 1e12)
+                                    >= step_bytes / (hbm_peak * 1e9) else "hbm"),
+                          "roofline_ms": step_t_roof * 1e3, "frac": step_t_roof * 1e3 / ms,
+                          "hbm_gbs": step_bytes / (ms * 1e-3) / 1e9,
+                          "algorithmic_bytes": step_bytes, "experts_touched": touched},
         "e2e": {"value": flops / (e2e * 1e-3) / 1e12, "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
         "gpu_launches": 6 * K,  # count+scan, scatter, permute, linear1, linear2, combine
