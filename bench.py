@@ -75,7 +75,7 @@ def _peaks():
 
 
 class ClockSampler:
-    """SM clock and clock-event reasons sampled through NVML every ~1 ms in a
+    """SM clock and clock-event reasons sampled through NVML every ~0.2 ms in a
     background thread while the timed region runs."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
@@ -119,7 +119,7 @@ class ClockSampler:
                 except Exception as e:
                     self.err = str(e)
                     return
-                time.sleep(0.001)
+                time.sleep(0.0002)
 
         self.thread = threading.Thread(target=loop, daemon=True)
         self.thread.start()
