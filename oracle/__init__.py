@@ -68,6 +68,9 @@ def _load():
         + [c_u8p, c_i32p, c_i32p, ctypes.POINTER(ctypes.c_float), c_u8p, c_u8p, c_u8p, c_u8p,
            c_i32p, ctypes.c_int, ctypes.POINTER(ctypes.c_uint16),
            ctypes.POINTER(ctypes.c_double), ctypes.c_int])
+    lib.orc_gemm.restype = None
+    lib.orc_gemm.argtypes = ([ctypes.c_int] * 4 + [c_u8p, c_i32p, c_i32p, c_u8p, c_u8p,
+                                                   ctypes.POINTER(ctypes.c_uint16), ctypes.c_int])
     lib.orc_max_threads.restype = ctypes.c_int
     lib.orc_max_threads.argtypes = []
     _lib = lib
@@ -182,6 +185,28 @@ def moe_forward(x, x_sf, topk_idx, topk_w, w1, w1_sf, w2, w2_sf, tokens=None,
         _ptr(y, ctypes.c_uint16),
         _ptr(acc, ctypes.c_double) if acc is not None else None, int(nthreads))
     return y, acc, bad
+
+
+def gemm(a, a_sf, b, b_sf, masked_m=None, out=None, nthreads=0):
+    """FP8 x FP4 GEMM, BF16 out (bits).  a u8 [G, M, K] (or [M, K]); a_sf i32
+    [G, M, K/128]; b u8 [G, N, K/2] (or [N, K/2]); b_sf u8 [G, N, K/32];
+    masked_m i32 [G] or None.  Rows at and beyond masked_m[g] keep the value
+    they have in `out` (zeros when `out` is None)."""
+    dense = a.ndim == 2
+    a3 = np.ascontiguousarray(a if not dense else a[None], np.uint8)
+    as3 = np.ascontiguousarray(a_sf if not dense else a_sf[None], np.int32)
+    b3 = np.ascontiguousarray(b if b.ndim == 3 else b[None], np.uint8)
+    bs3 = np.ascontiguousarray(b_sf if b_sf.ndim == 3 else b_sf[None], np.uint8)
+    G, M, K = a3.shape
+    N = b3.shape[1]
+    d = np.zeros((G, M, N), np.uint16) if out is None else np.ascontiguousarray(
+        out.reshape(G, M, N), np.uint16).copy()
+    mm = None if masked_m is None else np.ascontiguousarray(masked_m, np.int32)
+    _load().orc_gemm(G, M, N, K, _ptr(a3, ctypes.c_uint8), _ptr(as3, ctypes.c_int32),
+                     _ptr(mm, ctypes.c_int32) if mm is not None else None,
+                     _ptr(b3, ctypes.c_uint8), _ptr(bs3, ctypes.c_uint8),
+                     _ptr(d, ctypes.c_uint16), int(nthreads))
+    return d[0] if dense else d
 
 
 def max_threads() -> int:

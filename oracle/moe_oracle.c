@@ -305,6 +305,46 @@ int orc_moe_forward(int T, int H, int I, int E, int k, const uint8_t* x, const i
   return bad;
 }
 
+/* ------------------------------------------------------------------------ */
+/* FP8 x FP4 GEMM, dense and masked grouped ([EXPLAINER] 4.3: A FP8 [M, K]  */
+/* with block scales, B FP4 [N, K/2] packed with UE8M0 scales, D BF16;     */
+/* [OVERVIEW] 2 and [DAILY] "3. MoE模型专属优化": the masked grouped layout */
+/* for CUDA-graph decode, where only the device knows each group's rows).  */
+/* ------------------------------------------------------------------------ */
+/* Layouts: a u8 [G, M, K] E4M3, a_sf i32 [G, M, K/128] (byte j of word i =
+ * UE8M0 scale of K-block 4i+j, as x_sf), b u8 [G, N, K/2] E2M1 (low nibble
+ * = even k), b_sf u8 [G, N, K/32], d u16 [G, M, N] BF16 bits.
+ * D[g][m][n] = BF16_RNE( sum_k A[g][m][k] * B[g][n][k] ), decoded values,
+ * summed in double, for m < rows_g where rows_g = masked_m[g] (clamped to
+ * [0, M]) or M when masked_m is NULL.  Rows m >= rows_g are not written. */
+void orc_gemm(int G, int M, int N, int K, const uint8_t* a, const int32_t* a_sf,
+              const int32_t* masked_m, const uint8_t* b, const uint8_t* b_sf, uint16_t* d,
+              int nthreads) {
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+  for (int g = 0; g < G; ++g) {
+    int rows = masked_m ? masked_m[g] : M;
+    if (rows < 0) rows = 0;
+    if (rows > M) rows = M;
+    const uint8_t* ag = a + (size_t)g * M * K;
+    const int32_t* asg = a_sf + (size_t)g * M * (K / 128);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int m = 0; m < rows; ++m) {
+      double* ad = (double*)malloc(sizeof(double) * (size_t)K);
+      for (int kk = 0; kk < K; ++kk) ad[kk] = x_value(ag, asg, K, m, kk);
+      for (int n = 0; n < N; ++n) {
+        double sum = 0.0;
+        for (int kk = 0; kk < K; ++kk) sum += ad[kk] * w_value(b, b_sf, N, K, g, n, kk);
+        d[((size_t)g * M + m) * N + n] = orc_bf16_rne(sum);
+      }
+      free(ad);
+    }
+  }
+}
+
 int orc_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();
