@@ -401,9 +401,87 @@ def run_ours(args, wl, dist, rank, world, local_rank):
     print(json.dumps(out), flush=True)
 
 
+# ------------------------------------------------- standalone FP8 x FP4 GEMM
+GEMM_SHAPES = {"gemm": (4096, 7168, 7168), "gemm-small": (512, 2048, 1024)}
+
+
+def run_gemm(args, name):
+    """The standalone dense GEMM (one prefill-sized projection): K timed
+    replays of one captured call, L2 flushed before each, one JSON line."""
+    import numpy as np
+    import torch
+
+    import block_scaled_fp8_permute_b200 as moe
+    import synth
+
+    M, N, K = GEMM_SHAPES[name]
+    a, a_sf = synth.make_x(M, K, 0)
+    b, b_sf = synth.make_w(1, N, K, 2, 0)
+    dev = "cuda:0"
+    da = torch.from_numpy(a).to(dev)
+    das = torch.from_numpy(a_sf).to(dev)
+    b_t, b_sf_t = moe.gemm_transform_b(1, N, K, torch.from_numpy(b).to(dev),
+                                       torch.from_numpy(b_sf).to(dev))
+    d = torch.empty((M, N), dtype=torch.int16, device=dev)
+    ws = moe.alloc_gemm_workspace(1, M, N, K, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        moe.moe_gemm_fp8_fp4(M, N, K, da, das, b_t, b_sf_t, d, ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        call()
+    stream.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    K_ = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
+    with ClockSampler(0) as clk:
+        for i in range(K_):
+            flush.zero_()
+            ev[i][0].record(stream)
+            graph.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K_))
+    flops = 2.0 * M * N * K
+    pk = _peaks()
+    peak = 2.0 * pk["bf16"]
+    tflops = flops / (ms * 1e-3) / 1e12
+    algo_bytes = M * K + M * (K // 32) + N * K // 2 + N * (K // 32) + M * N * 2
+    del graph
+    print(json.dumps({
+        "metric": "FP8xFP4 GEMM TFLOPS on 1 B200 (standalone, BF16 out)", "value": tflops,
+        "unit": "TFLOPS", "n_gpus": 1, "steps": K_, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3 x fp4_e2m1, fp32 accumulate, bf16 out", "data": "synthetic",
+        "config": {"workload": f"{name}: M={M} N={N} K={K}", "l2": "flushed before every step",
+                   "step": "one moe_gemm_fp8_fp4 call replayed as a CUDA graph"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "kernel": "moe_gemm_kernel<3>",
+                     "flops_per_launch": flops, "algorithmic_bytes_per_launch": algo_bytes,
+                     "traffic": None,
+                     "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"},
+        "gpu_launches": 3 * K_,  # scale chunks + tile list, GEMM
+        "clocks": clk.summary(), "cpu_baseline": None}), flush=True)
+
+
 def main():
     args = _args()
     import synth
+    if args.workload in GEMM_SHAPES:
+        if int(os.environ.get("RANK", "0")) == 0 and args.impl == "ours":
+            run_gemm(args, args.workload)
+        return
     wl = synth.workload(args.workload)
     if args.impl == "reference":
         # the CPU oracle runs on rank 0 only; other ranks leave at once

@@ -64,6 +64,11 @@ _SIGS = {
     "moe_debug_requant": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
     "moe_set_timing_events": (None, [ctypes.POINTER(_vp), _i]),
     "moe_forward_noalloc": (_i, [_shp] + [_vp] * 9 + [_vp]),
+    "moe_gemm_b_bytes": (_sz, [_i, _i, _i, ctypes.POINTER(_sz)]),
+    "moe_gemm_transform_b": (_i, [_i, _i, _i] + [_vp] * 4 + [_vp]),
+    "moe_gemm_workspace_bytes": (_sz, [_i, _i, _i, _i]),
+    "moe_gemm_fp8_fp4": (_i, [_i, _i, _i] + [_vp] * 6 + [_sz, _vp]),
+    "moe_gemm_fp8_fp4_masked": (_i, [_i, _i, _i, _i] + [_vp] * 7 + [_sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -235,6 +240,38 @@ def moe_debug_requant(a, codes, sbytes, stream=None):
                                                        _ptr(sbytes), _stream(stream)))
 
 
+def moe_gemm_b_bytes(G: int, N: int, K: int):
+    sf = _sz(0)
+    n = _lib.moe_gemm_b_bytes(G, N, K, ctypes.byref(sf))
+    return n, sf.value
+
+
+def moe_gemm_transform_b(G, N, K, b, b_sf, b_t, b_sf_t, stream=None):
+    _check("moe_gemm_transform_b", _lib.moe_gemm_transform_b(
+        G, N, K, _ptr(b), _ptr(b_sf), _ptr(b_t), _ptr(b_sf_t), _stream(stream)))
+
+
+def moe_gemm_workspace_bytes(G: int, M_max: int, N: int, K: int) -> int:
+    return _lib.moe_gemm_workspace_bytes(G, M_max, N, K)
+
+
+def moe_gemm_fp8_fp4(M, N, K, a, a_sf, b_t, b_sf_t, d, workspace, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check("moe_gemm_fp8_fp4", _lib.moe_gemm_fp8_fp4(
+        M, N, K, _ptr(a), _ptr(a_sf), _ptr(b_t), _ptr(b_sf_t), _ptr(d), _ptr(workspace),
+        ws_bytes, _stream(stream)))
+
+
+def moe_gemm_fp8_fp4_masked(G, M_max, N, K, a, a_sf, masked_m, b_t, b_sf_t, d, workspace,
+                            ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check("moe_gemm_fp8_fp4_masked", _lib.moe_gemm_fp8_fp4_masked(
+        G, M_max, N, K, _ptr(a), _ptr(a_sf), _ptr(masked_m), _ptr(b_t), _ptr(b_sf_t), _ptr(d),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+
+
 # ------------------------------------------------------- torch conveniences
 def transform_weights(shp, w1, w1_sf, w2, w2_sf, stream=None):
     """Allocate the transformed weight buffers (torch, on w1's device) and
@@ -251,4 +288,20 @@ def transform_weights(shp, w1, w1_sf, w2, w2_sf, stream=None):
 def alloc_workspace(shp, device, host_variant=False):
     import torch
     n = moe_workspace_bytes_host(shp) if host_variant else moe_workspace_bytes(shp)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def gemm_transform_b(G, N, K, b, b_sf, stream=None):
+    """Allocate the transformed B buffers (torch, on b's device) and run
+    moe_gemm_transform_b.  Returns (b_t, b_sf_t)."""
+    import torch
+    n, sfn = moe_gemm_b_bytes(G, N, K)
+    outs = [torch.empty(max(v, 256), dtype=torch.uint8, device=b.device) for v in (n, sfn)]
+    moe_gemm_transform_b(G, N, K, b, b_sf, *outs, stream=stream)
+    return tuple(outs)
+
+
+def alloc_gemm_workspace(G, M_max, N, K, device):
+    import torch
+    n = moe_gemm_workspace_bytes(G, M_max, N, K)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)

@@ -30,6 +30,9 @@ cudaError_t launch_combine(const uint16_t* yp, const int* row_of, int T, int H, 
                            uint16_t* y, int grid, bool pdl, cudaStream_t stream);
 cudaError_t launch_transform(const uint8_t* w, const uint8_t* w_sf, int E, int N, int K,
                              int interleave, uint8_t* wt, uint8_t* wt_sf, cudaStream_t stream);
+cudaError_t launch_gemm_prep(const int* masked_m, int G, int m_max, int mt_per_g, int* tile_expert,
+                             int* norm_mtiles, int* hdr, const int32_t* a_sf, long long rows, int KG,
+                             uint8_t* sf_chunks, cudaStream_t stream);
 
 namespace {
 
@@ -162,6 +165,84 @@ struct Ws {
 };
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// standalone GEMM: shape rules and workspace (header, tile lists, A's scale chunks)
+moe_status check_gemm(int G, int M_max, int N, int K) {
+  if (G < 1 || M_max < 0 || N <= 0 || K <= 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (N % 128 || K % 128 || N > 65536 || K > 65536) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)G * M_max > (1LL << 24) || (long long)G * N * (K / 128) > (1LL << 31))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+struct GemmWs {
+  size_t hdr, tile_expert, norm_mt, sf, total;
+  int mt_per_g, MT;
+};
+GemmWs gemm_ws(int G, int M_max, int K) {
+  GemmWs w{};
+  w.mt_per_g = (M_max + kBlockM - 1) / kBlockM;
+  w.MT = G * w.mt_per_g;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  w.hdr = take(kHdrWords * 4);
+  w.tile_expert = take((size_t)w.MT * 4 + 4);
+  w.norm_mt = take((size_t)w.MT * 4 + 4);
+  w.sf = take((size_t)w.MT * (K / 128) * kSfChunk);
+  w.total = off;
+  return w;
+}
+
+moe_status gemm_run(int G, int M_max, int N, int K, const uint8_t* a, const int32_t* a_sf,
+                    const int32_t* masked_m, const void* b_t, const void* b_sf_t, uint16_t* d,
+                    void* workspace, size_t ws_bytes, cudaStream_t s) {
+  const GemmWs L = gemm_ws(G, M_max, K);
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  const long long rows = (long long)G * M_max;
+  if (rows == 0) return MOE_OK;
+  const void* p16[] = {a, a_sf, d};
+  for (const void* p : p16)
+    if (!p || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  if (!b_t || !b_sf_t || !aligned(b_t, 256) || !aligned(b_sf_t, 256)) return MOE_ERR_INVALID_ARG;
+  if (masked_m && !aligned(masked_m, 4)) return MOE_ERR_INVALID_ARG;
+  const int sms = device_sms();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  int* hdr = reinterpret_cast<int*>(base + L.hdr);
+  int* tile_expert = reinterpret_cast<int*>(base + L.tile_expert);
+  int* norm_mt = reinterpret_cast<int*>(base + L.norm_mt);
+  uint8_t* sf = base + L.sf;
+  const int KB = K / 128, NT = (N + kBlockN - 1) / kBlockN;
+  CUtensorMap tmA, tmB, tmD;
+  if (!encode_act(&tmA, a, (int)rows, K) || !encode_wgt(&tmB, b_t, G, KB, N, 256) ||
+      !encode_out_bf16(&tmD, d, (int)rows, N))
+    return MOE_ERR_CUDA;
+  cudaError_t e = cudaMemsetAsync(hdr, 0, kHdrWords * 4, s);
+  if (e == cudaSuccess)
+    e = launch_gemm_prep(masked_m, G, M_max, L.mt_per_g, tile_expert, norm_mt, hdr, a_sf, rows,
+                         KB, sf, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs g{};
+  g.sfa = sf;
+  g.sfb = static_cast<const uint8_t*>(b_sf_t);
+  g.hdr = hdr;
+  g.tile_expert = tile_expert;
+  g.norm_mtiles = norm_mt;
+  g.KB = KB;
+  g.n_rows = N;
+  g.NT = NT;
+  g.d = d;
+  g.masked_m = masked_m;
+  g.m_max = M_max;
+  const long long tiles = (long long)L.MT * NT;
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  return cuda_status(launch_gemm(3, tmA, tmB, tmD, g, grid < 1 ? 1 : grid, g_pdl.load() != 0, s));
+}
 
 // staging area of moe_forward_host, after the regular workspace
 struct HostStage {
@@ -488,6 +569,53 @@ moe_status moe_plan_export(const moe_shape* shape, const void* workspace, int32_
       return MOE_ERR_CUDA;
   }
   return MOE_OK;
+}
+
+size_t moe_gemm_b_bytes(int G, int N, int K, size_t* sf_bytes) {
+  if (check_gemm(G, 0, N, K) != MOE_OK) {
+    if (sf_bytes) *sf_bytes = 0;
+    return 0;
+  }
+  const size_t elems = (size_t)G * N * K;
+  if (sf_bytes) *sf_bytes = elems / 32;
+  return elems / 2;
+}
+
+moe_status moe_gemm_transform_b(int G, int N, int K, const uint8_t* b, const uint8_t* b_sf,
+                                void* b_t, void* b_sf_t, moe_stream_t stream) {
+  moe_status st = check_gemm(G, 0, N, K);
+  if (st != MOE_OK) return st;
+  if (!b || !b_sf || !aligned(b, 16) || !aligned(b_sf, 16)) return MOE_ERR_INVALID_ARG;
+  if (!b_t || !b_sf_t || !aligned(b_t, 256) || !aligned(b_sf_t, 256)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_transform(b, b_sf, G, N, K, 0, static_cast<uint8_t*>(b_t),
+                                      static_cast<uint8_t*>(b_sf_t),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t moe_gemm_workspace_bytes(int G, int M_max, int N, int K) {
+  if (check_gemm(G, M_max, N, K) != MOE_OK) return 0;
+  return gemm_ws(G, M_max, K).total;
+}
+
+moe_status moe_gemm_fp8_fp4(int M, int N, int K, const uint8_t* a, const int32_t* a_sf,
+                            const void* b_t, const void* b_sf_t, uint16_t* d, void* workspace,
+                            size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_gemm(1, M, N, K);
+  if (st != MOE_OK) return st;
+  return gemm_run(1, M, N, K, a, a_sf, nullptr, b_t, b_sf_t, d, workspace, ws_bytes,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_gemm_fp8_fp4_masked(int G, int M_max, int N, int K, const uint8_t* a,
+                                   const int32_t* a_sf, const int32_t* masked_m, const void* b_t,
+                                   const void* b_sf_t, uint16_t* d, void* workspace,
+                                   size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_gemm(G, M_max, N, K);
+  if (st != MOE_OK) return st;
+  if (M_max % kBlockM) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!masked_m) return MOE_ERR_INVALID_ARG;
+  return gemm_run(G, M_max, N, K, a, a_sf, masked_m, b_t, b_sf_t, d, workspace, ws_bytes,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_debug_requant(const float* a, int rows, int cols, uint8_t* codes, uint8_t* sbytes,

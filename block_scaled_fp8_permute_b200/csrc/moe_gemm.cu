@@ -5,7 +5,9 @@
 //            UE8M0 scale per 1x32 block on both sides, FP32 accumulation) with
 //            the SwiGLU + E4M3 requantisation epilogue fused in;
 //   linear2: O = A2_e . W2_e^T with the top-k weight applied in the epilogue,
-//            BF16 partial rows written in expert-contiguous row order.
+//            BF16 partial rows written in expert-contiguous row order;
+//   the standalone FP8 x FP4 GEMM (dense or masked grouped): D = A_g . B_g^T,
+//            BF16 rows.
 // ("DeepSeek DeepGEMM 2026年4月重磅更新：Mega MoE融合算子、FP4精度与极致性能优化",
 //  section 3.2 (fusing linear1 / SwiGLU / linear2), section 4.2 (UE8M0 scale
 //  factors, FP32 accumulation), section 11.3 (TMA multi-stage loads).)
@@ -63,7 +65,8 @@ __global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int 
 }
 
 // -------------------------------------------------------------------- kernel
-template <int kEpi>  // 1: SwiGLU + requant (linear1), 2: x topk_w, BF16 rows (linear2)
+template <int kEpi>  // 1: SwiGLU + requant (linear1), 2: x topk_w, BF16 rows (linear2),
+                     // 3: BF16 rows of the standalone GEMM
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    if (kEpi == 2) prefetch_tmap(&tmOut);
+    if (kEpi != 1) prefetch_tmap(&tmOut);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, kTmemCols);
@@ -237,7 +240,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) mbar_arrive(acc_empty);
       epilogue_store<kEpi>(v, args, &tmOut, sOut + ew * kOutStage, mt, nt, r, h, q, lane);
     }
-    if (kEpi == 2 && lane == 0) bulk_wait_group0();  // stores complete before the CTA exits
+    if (kEpi != 1 && lane == 0) bulk_wait_group0();  // stores complete before the CTA exits
   }
 
   pdl_launch();
@@ -254,9 +257,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmOut, const GemmArgs& args, int grid, bool pdl,
                         cudaStream_t stream) {
-  static bool attr_set[3] = {false, false, false};
+  static bool attr_set[4] = {false, false, false, false};
   void (*fn)(CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs) =
-      (epi == 1) ? moe_gemm_kernel<1> : moe_gemm_kernel<2>;
+      (epi == 1) ? moe_gemm_kernel<1> : (epi == 2 ? moe_gemm_kernel<2> : moe_gemm_kernel<3>);
   if (!attr_set[epi]) {
     cudaError_t err = cudaFuncSetAttribute((const void*)fn,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -108,6 +108,11 @@ struct GemmArgs {
   const int* swap_experts; // experts with swapped operand roles
   const int* poffs;        // padded first row of every expert
   const int* counts;       // rows of every expert
+  // standalone GEMM (epilogue 3): D rows [G * m_max, n_rows] BF16; group g of an
+  // m-tile = tile_expert[mt]; rows at and past masked_m[g] (m_max when NULL) are not written
+  uint16_t* d;
+  const int* masked_m;
+  int m_max;
 };
 
 // experts with at most this many routed rows use swapped operand roles

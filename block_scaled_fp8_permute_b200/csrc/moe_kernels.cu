@@ -259,6 +259,84 @@ __global__ void combine_kernel(const uint16_t* __restrict__ yp, const int* __res
   pdl_launch_k();
 }
 
+// ------------------------------------------------------- standalone GEMM
+// Tile lists of the FP8 x FP4 GEMM (dense or masked grouped): group g owns
+// m-tiles g*mt_per_g .. g*mt_per_g + ceil(rows_g / 128) - 1 with rows_g =
+// masked_m[g] (m_max when masked_m is NULL), read on the device so a
+// captured graph follows the counts of each replay.  One block of 1024.
+__global__ void __launch_bounds__(1024) gemm_plan_kernel(const int* __restrict__ masked_m, int G,
+                                                         int m_max, int mt_per_g,
+                                                         int* __restrict__ tile_expert,
+                                                         int* __restrict__ norm_mtiles,
+                                                         int* __restrict__ hdr) {
+  __shared__ int wsum[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int g0 = 0; g0 < G; g0 += blockDim.x) {
+    const int g = g0 + tid;
+    int c = 0;
+    if (g < G) {
+      int rows = masked_m ? masked_m[g] : m_max;
+      if (rows < 0 || rows > m_max) {
+        set_status(hdr, MOE_ERR_INVALID_ARG);
+        rows = rows < 0 ? 0 : m_max;
+      }
+      c = (rows + kBlockM - 1) / kBlockM;
+      for (int i = 0; i < mt_per_g; ++i) tile_expert[(size_t)g * mt_per_g + i] = g;
+    }
+    int incl = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += t;
+    }
+    if (lane == 31) wsum[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+      int w = wsum[lane];
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, w, d);
+        if (lane >= d) w += t;
+      }
+      wsum[lane] = w;
+    }
+    __syncthreads();
+    const int pre = carry + (wid ? wsum[wid - 1] : 0) + incl - c;
+    for (int i = 0; i < c; ++i) norm_mtiles[pre + i] = g * mt_per_g + i;
+    __syncthreads();
+    if (tid == 0) carry += wsum[31];
+    __syncthreads();
+  }
+  if (tid == 0) hdr[kHdrNormMTiles] = carry;
+}
+
+// A's scale words [rows][KG] into the 512-byte chunks the GEMM streams.
+__global__ void sf_chunks_kernel(const int32_t* __restrict__ a_sf, long long rows, int KG,
+                                 uint8_t* __restrict__ out) {
+  const long long n = rows * KG;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / KG), kg = (int)(i - (long long)r * KG);
+    *reinterpret_cast<int32_t*>(out + sf_chunk_offset(r, kg, KG)) = a_sf[i];
+  }
+}
+
+cudaError_t launch_gemm_prep(const int* masked_m, int G, int m_max, int mt_per_g, int* tile_expert,
+                             int* norm_mtiles, int* hdr, const int32_t* a_sf, long long rows, int KG,
+                             uint8_t* sf_chunks, cudaStream_t stream) {
+  gemm_plan_kernel<<<1, 1024, 0, stream>>>(masked_m, G, m_max, mt_per_g, tile_expert, norm_mtiles,
+                                           hdr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || rows == 0) return e;
+  long long grid = (rows * KG + 255) / 256;
+  if (grid > 148LL * 16) grid = 148LL * 16;
+  sf_chunks_kernel<<<(unsigned)grid, 256, 0, stream>>>(a_sf, rows, KG, sf_chunks);
+  return cudaGetLastError();
+}
+
 // -------------------------------------------------------------- transform
 // One thread per (expert, K-block, transformed row): 64 bytes of codes and
 // one 32-bit word of scales.  interleave != 0 applies the W1 gate/up

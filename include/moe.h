@@ -243,6 +243,52 @@ void moe_set_timing_events(void* const* events, int n);
 moe_status moe_debug_requant(const float* a, int rows, int cols, uint8_t* codes, uint8_t* sbytes,
                              moe_stream_t stream);
 
+/* ------------------------------------------------- standalone FP8 x FP4 GEMM */
+/* D = A . B^T with A FP8 E4M3 [M, K] (one UE8M0 scale per 1x32 block, four
+ * per int32 as x_sf), B FP4 E2M1 [N, K/2] (low nibble = even k, one UE8M0
+ * byte per 1x32 block) and D BF16 [M, N], FP32 accumulation, one BF16
+ * rounding ("DeepSeek DeepGEMM 2026年4月重磅更新" section 4.3, the
+ * fp8_fp4_gemm call).  The masked grouped form computes G such products
+ * with A [G, M_max, K], B [G, N, K/2], D [G, M_max, N], where only rows
+ * m < masked_m[g] of group g are computed and written; masked_m lives on
+ * the device, so a captured CUDA graph follows the counts of each replay
+ * (the masked layout for CUDA-graph decode: "DeepGEMM: DeepSeek
+ * 把大模型核心算子打包成一座 CUDA 训练场" section 2).  Same tensor-core
+ * kernel as the MoE layer's linears.
+ *
+ * Shapes: N and K multiples of 128 (N, K <= 65536), G >= 1, G * M_max <=
+ * 2^24; the masked form needs M_max % 128 == 0; the dense form takes any
+ * M >= 0.  Errors: MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_INVALID_ARG (NULL or
+ * misaligned pointer: A, A scales and D 16-byte aligned; transformed B and
+ * the workspace 256-byte aligned), MOE_ERR_WORKSPACE; a masked_m value
+ * outside [0, M_max] is clamped on the device and reported as
+ * MOE_ERR_INVALID_ARG by moe_get_device_status(workspace).  All pointers
+ * are caller-owned device memory; calls are enqueued on `stream`. */
+
+/* Bytes of B after moe_gemm_transform_b (codes; *sf_bytes: scales), 0 for
+ * an unsupported shape. */
+size_t moe_gemm_b_bytes(int G, int N, int K, size_t* sf_bytes);
+
+/* One-time repack of B (G groups, canonical layout above) into the
+ * K-block-major layout and 512-byte scale chunks the kernel streams (the
+ * layout moe_transform_weights gives W2). */
+moe_status moe_gemm_transform_b(int G, int N, int K, const uint8_t* b, const uint8_t* b_sf,
+                                void* b_t, void* b_sf_t, moe_stream_t stream);
+
+/* Workspace bytes of one call (tile lists and A's scale chunks), 0 for an
+ * unsupported shape.  For the dense form pass G = 1, M_max = M. */
+size_t moe_gemm_workspace_bytes(int G, int M_max, int N, int K);
+
+moe_status moe_gemm_fp8_fp4(int M, int N, int K, const uint8_t* a, const int32_t* a_sf,
+                            const void* b_t, const void* b_sf_t, uint16_t* d, void* workspace,
+                            size_t ws_bytes, moe_stream_t stream);
+
+/* masked_m: device int32 [G]. */
+moe_status moe_gemm_fp8_fp4_masked(int G, int M_max, int N, int K, const uint8_t* a,
+                                   const int32_t* a_sf, const int32_t* masked_m, const void* b_t,
+                                   const void* b_sf_t, uint16_t* d, void* workspace,
+                                   size_t ws_bytes, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -104,3 +104,33 @@ def test_zero_tokens_is_a_no_op(moe):
     st = moe.lib().moe_forward(ctypes.byref(s), None, None, None, None, 256, 256, 256, 256, None,
                                4096, ws, None)
     assert st == 0
+
+
+def test_gemm_sizes_and_validation(moe):
+    lib = moe.lib()
+    assert moe.moe_gemm_b_bytes(2, 256, 512) == (2 * 256 * 512 // 2, 2 * 256 * 512 // 32)
+    assert moe.moe_gemm_b_bytes(1, 100, 512)[0] == 0          # N % 128
+    ws = moe.moe_gemm_workspace_bytes(1, 300, 256, 512)
+    # at least A's scale chunks: 3 m-tiles x 4 K-blocks x 512 bytes
+    assert ws >= 3 * 4 * 512
+    assert moe.moe_gemm_workspace_bytes(1, 300, 256, 500) == 0  # K % 128
+    assert moe.moe_gemm_workspace_bytes(0, 128, 256, 512) == 0  # no group
+    ok = [256, 256, 256, 256, 256]                              # a, a_sf, b_t, b_sf_t, d
+    # unsupported shapes
+    assert lib.moe_gemm_fp8_fp4(300, 200, 512, *ok, 4096, ws, None) == 2
+    assert lib.moe_gemm_fp8_fp4_masked(2, 100, 256, 512, 256, 256, 256, 256, 256, 256,
+                                       4096, ws, None) == 2   # M_max % 128
+    # masked form without counts
+    assert lib.moe_gemm_fp8_fp4_masked(2, 128, 256, 512, 256, 256, None, 256, 256, 256,
+                                       4096, ws, None) == 1
+    # workspace: null, misaligned, too small
+    assert lib.moe_gemm_fp8_fp4(300, 256, 512, *ok, None, ws, None) == 1
+    assert lib.moe_gemm_fp8_fp4(300, 256, 512, *ok, 4096 + 64, ws, None) == 1
+    assert lib.moe_gemm_fp8_fp4(300, 256, 512, *ok, 4096, 16, None) == 3
+    # operands: null / misaligned A, B not 256-byte aligned
+    assert lib.moe_gemm_fp8_fp4(300, 256, 512, None, 256, 256, 256, 256, 4096, ws, None) == 1
+    assert lib.moe_gemm_fp8_fp4(300, 256, 512, 256 + 4, 256, 256, 256, 256, 4096, ws, None) == 1
+    assert lib.moe_gemm_fp8_fp4(300, 256, 512, 256, 256, 256 + 16, 256, 256, 4096, ws, None) == 1
+    # no rows: nothing to do
+    ws0 = moe.moe_gemm_workspace_bytes(1, 0, 256, 512)
+    assert lib.moe_gemm_fp8_fp4(0, 256, 512, None, None, None, None, None, 4096, ws0, None) == 0
