@@ -402,33 +402,42 @@ def run_ours(args, wl, dist, rank, world, local_rank):
 
 
 # ------------------------------------------------- standalone FP8 x FP4 GEMM
-GEMM_SHAPES = {"gemm": (4096, 7168, 7168), "gemm-small": (512, 2048, 1024)}
+# name -> (G, M or M_max, N, K, masked): a prefill-sized dense projection, a small one,
+# and a decode-style masked grouped GEMM (16 groups, 1..64 rows each, weights read once)
+GEMM_SHAPES = {"gemm": (1, 4096, 7168, 7168, False), "gemm-small": (1, 512, 2048, 1024, False),
+               "gemm-masked": (16, 128, 4096, 7168, True)}
 
 
 def run_gemm(args, name):
-    """The standalone dense GEMM (one prefill-sized projection): K timed
-    replays of one captured call, L2 flushed before each, one JSON line."""
+    """The standalone GEMM: K timed replays of one captured call, L2 flushed
+    before each, one JSON line."""
     import numpy as np
     import torch
 
     import block_scaled_fp8_permute_b200 as moe
     import synth
 
-    M, N, K = GEMM_SHAPES[name]
-    a, a_sf = synth.make_x(M, K, 0)
-    b, b_sf = synth.make_w(1, N, K, 2, 0)
+    G, M, N, K, masked = GEMM_SHAPES[name]
+    a, a_sf = synth.make_x(G * M, K, 0)
+    b, b_sf = synth.make_w(G, N, K, 2, 0)
+    counts = (np.random.default_rng(0).integers(1, 65, G).astype(np.int32) if masked
+              else np.full(G, M, np.int32))
     dev = "cuda:0"
     da = torch.from_numpy(a).to(dev)
     das = torch.from_numpy(a_sf).to(dev)
-    b_t, b_sf_t = moe.gemm_transform_b(1, N, K, torch.from_numpy(b).to(dev),
+    b_t, b_sf_t = moe.gemm_transform_b(G, N, K, torch.from_numpy(b).to(dev),
                                        torch.from_numpy(b_sf).to(dev))
-    d = torch.empty((M, N), dtype=torch.int16, device=dev)
-    ws = moe.alloc_gemm_workspace(1, M, N, K, dev)
+    d = torch.empty((G * M, N), dtype=torch.int16, device=dev)
+    mm = torch.from_numpy(counts).to(dev)
+    ws = moe.alloc_gemm_workspace(G, M, N, K, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def call():
-        moe.moe_gemm_fp8_fp4(M, N, K, da, das, b_t, b_sf_t, d, ws)
+        if masked:
+            moe.moe_gemm_fp8_fp4_masked(G, M, N, K, da, das, mm, b_t, b_sf_t, d, ws)
+        else:
+            moe.moe_gemm_fp8_fp4(M, N, K, da, das, b_t, b_sf_t, d, ws)
 
     side = torch.cuda.Stream()
     side.wait_stream(stream)
@@ -453,25 +462,32 @@ def run_gemm(args, name):
             ev[i][1].record(stream)
         torch.cuda.synchronize()
     ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K_))
-    flops = 2.0 * M * N * K
+    rows = int(counts.sum())
+    flops = 2.0 * rows * N * K
+    algo_bytes = (rows * (K + K // 32) + G * (N * K // 2 + N * (K // 32)) + rows * N * 2)
     pk = _peaks()
-    peak = 2.0 * pk["bf16"]
+    tpeak, hpeak = 2.0 * pk["bf16"], pk["hbm"]
     tflops = flops / (ms * 1e-3) / 1e12
-    algo_bytes = M * K + M * (K // 32) + N * K // 2 + N * (K // 32) + M * N * 2
+    gbs = algo_bytes / (ms * 1e-3) / 1e9
+    if flops / (tpeak * 1e12) >= algo_bytes / (hpeak * 1e9):
+        roof = {"bound": "tensor", "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s",
+                "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hpeak, "unit": "GB/s",
+                "peak_note": f"copy bandwidth {hpeak} GB/s ({pk['src']})"}
+    roof.update(frac=roof["achieved"] / roof["peak"], kernel="moe_gemm_kernel<3>",
+                flops_per_launch=flops, algorithmic_bytes_per_launch=algo_bytes, traffic=None)
     del graph
+    shape = (f"G={G} M_max={M} (rows {rows}) N={N} K={K}" if masked else f"M={M} N={N} K={K}")
     print(json.dumps({
         "metric": "FP8xFP4 GEMM TFLOPS on 1 B200 (standalone, BF16 out)", "value": tflops,
-        "unit": "TFLOPS", "n_gpus": 1, "steps": K_, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "unit": "TFLOPS", "gbs": gbs, "n_gpus": 1, "steps": K_, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3 x fp4_e2m1, fp32 accumulate, bf16 out", "data": "synthetic",
-        "config": {"workload": f"{name}: M={M} N={N} K={K}", "l2": "flushed before every step",
-                   "step": "one moe_gemm_fp8_fp4 call replayed as a CUDA graph"},
-        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": tflops / peak, "kernel": "moe_gemm_kernel<3>",
-                     "flops_per_launch": flops, "algorithmic_bytes_per_launch": algo_bytes,
-                     "traffic": None,
-                     "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"},
-        "gpu_launches": 3 * K_,  # scale chunks + tile list, GEMM
+        "config": {"workload": f"{name}: {shape}", "l2": "flushed before every step",
+                   "step": "one GEMM call replayed as a CUDA graph"},
+        "roofline": roof,
+        "gpu_launches": 3 * K_,  # tile list, scale chunks, GEMM
         "clocks": clk.summary(), "cpu_baseline": None}), flush=True)
 
 
