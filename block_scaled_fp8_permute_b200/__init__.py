@@ -51,6 +51,7 @@ _SIGS = {
     "moe_set_pdl": (None, [_i]),
     "moe_set_gemm_variant": (None, [_i]),
     "moe_set_swap_max": (None, [_i]),
+    "moe_set_narrow_tiles": (None, [_i]),
     "moe_transformed_bytes": (_sz, [_shp, _i, ctypes.POINTER(_sz)]),
     "moe_transform_weights": (_i, [_shp] + [_vp] * 8 + [_vp]),
     "moe_workspace_bytes": (_sz, [_shp]),
@@ -133,6 +134,10 @@ def moe_set_gemm_variant(variant: int) -> None:
 
 def moe_set_swap_max(rows: int) -> None:
     _lib.moe_set_swap_max(rows)
+
+
+def moe_set_narrow_tiles(mode: int) -> None:
+    _lib.moe_set_narrow_tiles(mode)
 
 
 def moe_transformed_bytes(shp: MoeShape, which: int):

@@ -8,7 +8,7 @@
 #include "moe_internal.cuh"
 
 namespace moe {
-cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+cudaError_t launch_gemm(int epi, bool narrow, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmOut, const GemmArgs& args, int grid, bool pdl,
                         cudaStream_t stream);
 cudaError_t launch_gemm_pair(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
@@ -17,10 +17,10 @@ cudaError_t launch_gemm_pair(int epi, const CUtensorMap& tmA, const CUtensorMap&
                              bool pdl, cudaStream_t stream);
 cudaError_t launch_requant_debug(const float* a, int rows, int cols, uint8_t* codes,
                                  uint8_t* sbytes, cudaStream_t stream);
-cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max, int* chunk,
-                        int* counts, int* offs, int* poffs, int* tile_expert, int* mpair,
-                        int* norm_mtiles, int* swap_experts, int* row_of, int* src_of, int* hdr,
-                        bool pdl, cudaStream_t stream);
+cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max, int narrow_max,
+                        int* chunk, int* counts, int* offs, int* poffs, int* tile_expert,
+                        int* mpair, int* norm_mtiles, int* swap_experts, int* narrow_mtiles,
+                        int* row_of, int* src_of, int* hdr, bool pdl, cudaStream_t stream);
 cudaError_t launch_gemm_swap(int epi, const CUtensorMap& tmW, const CUtensorMap& tmX,
                              const GemmArgs& args, int grid, bool pdl, cudaStream_t stream);
 cudaError_t launch_permute(const uint8_t* x, const int32_t* x_sf, const int* src_of,
@@ -40,6 +40,7 @@ std::atomic<int> g_num_sms_cap{0};
 std::atomic<int> g_pdl{1};
 std::atomic<int> g_gemm_variant{0};
 std::atomic<int> g_swap_max{0};
+std::atomic<int> g_narrow_mode{-1};
 std::mutex g_ev_mu;
 cudaEvent_t g_events[5];
 bool g_events_on = false;
@@ -157,6 +158,7 @@ struct Ws {
   int* mpair() const { return reinterpret_cast<int*>(base + L.mpair); }
   int* norm_mt() const { return reinterpret_cast<int*>(base + L.norm_mt); }
   int* swap_e() const { return reinterpret_cast<int*>(base + L.swap_e); }
+  int* narrow_mt() const { return reinterpret_cast<int*>(base + L.narrow_mt); }
   uint8_t* xp() const { return base + L.xp; }
   uint8_t* xp_sf() const { return base + L.xp_sf; }
   uint8_t* a2() const { return base + L.a2; }
@@ -165,6 +167,18 @@ struct Ws {
 };
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Narrow-tile threshold of a shape, the same in moe_plan and moe_forward: on
+// (experts with 1..kNarrowRows rows) with one-SM tiles when the layer has at
+// most 128 rows per expert on average (decode-sized and fine-grained layers),
+// or always / never when set so; off with SM-pair tiles.
+int narrow_max_for(const moe_shape& s) {
+  if (g_gemm_variant.load() == 1) return 0;
+  const int mode = g_narrow_mode.load();
+  if (mode == 0) return 0;
+  if (mode < 0 && (long long)s.T * s.topk > (long long)kBlockM * s.E) return 0;
+  return kNarrowRows;
+}
 
 // standalone GEMM: shape rules and workspace (header, tile lists, A's scale chunks)
 moe_status check_gemm(int G, int M_max, int N, int K) {
@@ -233,6 +247,7 @@ moe_status gemm_run(int G, int M_max, int N, int K, const uint8_t* a, const int3
   g.hdr = hdr;
   g.tile_expert = tile_expert;
   g.norm_mtiles = norm_mt;
+  g.tiles_word = kHdrNormMTiles;
   g.KB = KB;
   g.n_rows = N;
   g.NT = NT;
@@ -241,7 +256,8 @@ moe_status gemm_run(int G, int M_max, int N, int K, const uint8_t* a, const int3
   g.m_max = M_max;
   const long long tiles = (long long)L.MT * NT;
   const int grid = (int)(tiles < sms ? tiles : sms);
-  return cuda_status(launch_gemm(3, tmA, tmB, tmD, g, grid < 1 ? 1 : grid, g_pdl.load() != 0, s));
+  return cuda_status(
+      launch_gemm(3, false, tmA, tmB, tmD, g, grid < 1 ? 1 : grid, g_pdl.load() != 0, s));
 }
 
 // staging area of moe_forward_host, after the regular workspace
@@ -292,6 +308,8 @@ void moe_set_num_sms(int num_sms) { g_num_sms_cap.store(num_sms > 0 ? num_sms : 
 void moe_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
 
 void moe_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }
+
+void moe_set_narrow_tiles(int mode) { g_narrow_mode.store(mode < 0 ? -1 : (mode ? 1 : 0)); }
 
 void moe_set_swap_max(int rows) {
   g_swap_max.store(rows < 0 ? 0 : (rows > kMaxSwapRows ? kMaxSwapRows : rows));
@@ -356,10 +374,10 @@ moe_status moe_plan(const moe_shape* shape, const int32_t* topk_idx, void* works
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(ws.hdr(), 0, kHdrWords * 4, s);
   if (e == cudaSuccess)
-    e = launch_plan(topk_idx, ws.L.R, shape->E, ws.L.NCH, g_swap_max.load(), ws.chunk(),
-                    ws.counts(), ws.offs(), ws.poffs(), ws.tile_expert(), ws.mpair(),
-                    ws.norm_mt(), ws.swap_e(), ws.row_of(), ws.src_of(), ws.hdr(),
-                    g_pdl.load() != 0, s);
+    e = launch_plan(topk_idx, ws.L.R, shape->E, ws.L.NCH, g_swap_max.load(),
+                    narrow_max_for(*shape), ws.chunk(), ws.counts(), ws.offs(), ws.poffs(),
+                    ws.tile_expert(), ws.mpair(), ws.norm_mt(), ws.swap_e(), ws.narrow_mt(),
+                    ws.row_of(), ws.src_of(), ws.hdr(), g_pdl.load() != 0, s);
   return cuda_status(e);
 }
 
@@ -395,6 +413,10 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   const bool pair2 = pair1 && (sh.H % 256) == 0;
   CUtensorMap tmX, tmW1, tmA2, tmW2, tmYp, tmXsf, tmW1sf, tmA2sf, tmW2sf;
   CUtensorMap tmX16, tmA216, tmW1s, tmW2s;  // swapped-role kernel: 16-row token boxes
+  CUtensorMap tmXn, tmA2n;                   // narrow tiles: kNarrowRows-row A boxes
+  if (!encode_act(&tmXn, ws.xp(), ws.L.P_max, sh.H, kNarrowRows) ||
+      !encode_act(&tmA2n, ws.a2(), ws.L.P_max, sh.I, kNarrowRows))
+    return MOE_ERR_CUDA;
   if (!encode_act(&tmX16, ws.xp(), ws.L.P_max, sh.H, 16) ||
       !encode_act(&tmA216, ws.a2(), ws.L.P_max, sh.I, 16) ||
       !encode_wgt(&tmW1s, w1_t, sh.E, KB1, 2 * sh.I, 256) ||
@@ -430,6 +452,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   g1.src_of = ws.src_of();
   g1.mpair = ws.mpair();
   g1.norm_mtiles = ws.norm_mt();
+  g1.tiles_word = kHdrNormMTiles;
   g1.swap_experts = ws.swap_e();
   g1.poffs = ws.poffs();
   g1.counts = ws.counts();
@@ -447,9 +470,19 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   } else {
     long long tiles1 = (long long)ws.L.MT_max * NT1;
     int grid1 = (int)(tiles1 < sms ? tiles1 : sms);
-    e = launch_gemm(1, tmX, tmW1, tmYp, g1, grid1 < 1 ? 1 : grid1, pdl, s);
+    e = launch_gemm(1, false, tmX, tmW1, tmYp, g1, grid1 < 1 ? 1 : grid1, pdl, s);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  // experts with at most kNarrowRows rows: narrow tiles (a deeper weight stream)
+  const bool narrow = narrow_max_for(sh) > 0;
+  const int narrow_grid1 = (int)((long long)sh.E * NT1 < sms ? (long long)sh.E * NT1 : sms);
+  if (narrow) {
+    GemmArgs g1n = g1;
+    g1n.norm_mtiles = ws.narrow_mt();
+    g1n.tiles_word = kHdrNarrowMTiles;
+    e = launch_gemm(1, true, tmXn, tmW1, tmYp, g1n, narrow_grid1, pdl, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
   // swapped-role tiles exist only when the plan was made with a threshold > 0
   const bool use_swap = g_swap_max.load() > 0;
   if (use_swap) {
@@ -474,9 +507,17 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   } else {
     long long tiles2 = (long long)ws.L.MT_max * NT2;
     int grid2 = (int)(tiles2 < sms ? tiles2 : sms);
-    e = launch_gemm(2, tmA2, tmW2, tmYp, g2, grid2 < 1 ? 1 : grid2, pdl, s);
+    e = launch_gemm(2, false, tmA2, tmW2, tmYp, g2, grid2 < 1 ? 1 : grid2, pdl, s);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  if (narrow) {
+    GemmArgs g2n = g2;
+    g2n.norm_mtiles = ws.narrow_mt();
+    g2n.tiles_word = kHdrNarrowMTiles;
+    const int narrow_grid2 = (int)((long long)sh.E * NT2 < sms ? (long long)sh.E * NT2 : sms);
+    e = launch_gemm(2, true, tmA2n, tmW2, tmYp, g2n, narrow_grid2, pdl, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
   if (use_swap) {
     const int swap_grid2 = (int)((long long)sh.E * NT2 < sms ? (long long)sh.E * NT2 : sms);
     e = launch_gemm_swap(2, tmW2s, tmA216, g2, swap_grid2, pdl, s);

@@ -31,8 +31,6 @@
 
 namespace moe {
 
-constexpr int kStages = 4;
-constexpr int kSmemA = kBlockM * kBlockK;  // 16384 bytes
 constexpr int kSmemB = kBlockN * kBlockK;  // 32768 bytes (one byte per E2M1 element in smem)
 constexpr int kTxB = kBlockN * kBlockK / 2;  // bytes the TMA moves for B (packed)
 constexpr int kSmemSFA = kSfChunk;
@@ -43,8 +41,24 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;    // FP32 accumulator, 256 columns
 constexpr uint32_t kSfCol = 256;   // scale buffers: buf b -> SFA at +16b (4 cols), SFB at +16b+4 (8)
 constexpr int kOutStage = kEpiOutStage;
-constexpr size_t kGemmSmemBytes = 1024 + (size_t)kStages * (kSmemA + kSmemB + kSmemSFA + kSmemSFB) +
-                                  (size_t)kNumEpiWarps * kOutStage + 256;
+
+// Stage geometry.  Normal tiles stage 128 A rows (16 KB) per 128-K step in a
+// 4-deep ring.  Narrow tiles (experts with at most kNarrowRows rows: decode-
+// sized batches) stage only kNarrowRows A rows, and the 12 KB saved per stage
+// buy a fifth stage, i.e. 25 % more weight bytes in flight per SM.  The MMA
+// still spans 128 rows: rows past kNarrowRows read whatever the shared memory
+// after the stage's A rows holds, and those accumulator rows (padding) are
+// never stored.
+template <bool kNarrow>
+struct TileCfg {
+  static constexpr int kARows = kNarrow ? kNarrowRows : kBlockM;
+  static constexpr int kStages = kNarrow ? 5 : 4;
+  static constexpr int kSmemA = kARows * kBlockK;
+  static constexpr size_t kSmemBytes =
+      1024 + (size_t)kStages * (kSmemA + kSmemB + kSmemSFA + kSmemSFB) +
+      (size_t)kNumEpiWarps * kOutStage + 256;
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
 
 __global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int cols,
                                      uint8_t* __restrict__ codes, uint8_t* __restrict__ sbytes) {
@@ -65,13 +79,16 @@ __global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int 
 }
 
 // -------------------------------------------------------------------- kernel
-template <int kEpi>  // 1: SwiGLU + requant (linear1), 2: x topk_w, BF16 rows (linear2),
-                     // 3: BF16 rows of the standalone GEMM
+template <int kEpi,    // 1: SwiGLU + requant (linear1), 2: x topk_w, BF16 rows (linear2),
+                       // 3: BF16 rows of the standalone GEMM
+          bool kNarrow>  // stage only kNarrowRows A rows (TileCfg)
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmOut, const GemmArgs args) {
   using namespace ptx;
+  constexpr int kStages = TileCfg<kNarrow>::kStages;
+  constexpr int kSmemA = TileCfg<kNarrow>::kSmemA;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<size_t>(smem_raw), 1024));
   uint8_t* sA = smem;
@@ -115,7 +132,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   pdl_wait();  // inputs come from the previous kernel of the forward
   const int NT = args.NT, KB = args.KB, n_rows = args.n_rows;
-  const int num_tiles = args.hdr[kHdrNormMTiles] * NT;
+  const int num_tiles = args.hdr[args.tiles_word] * NT;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -254,23 +271,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ------------------------------------------------------------ host launchers
-cudaError_t launch_gemm(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
+cudaError_t launch_gemm(int epi, bool narrow, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         const CUtensorMap& tmOut, const GemmArgs& args, int grid, bool pdl,
                         cudaStream_t stream) {
-  static bool attr_set[4] = {false, false, false, false};
-  void (*fn)(CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs) =
-      (epi == 1) ? moe_gemm_kernel<1> : (epi == 2 ? moe_gemm_kernel<2> : moe_gemm_kernel<3>);
-  if (!attr_set[epi]) {
-    cudaError_t err = cudaFuncSetAttribute((const void*)fn,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)kGemmSmemBytes);
+  typedef void (*Fn)(CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs);
+  static bool attr_set[2][4] = {};
+  Fn fn;
+  size_t smem;
+  if (narrow) {
+    if (epi != 1 && epi != 2) return cudaErrorInvalidValue;
+    fn = epi == 1 ? moe_gemm_kernel<1, true> : moe_gemm_kernel<2, true>;
+    smem = TileCfg<true>::kSmemBytes;
+  } else {
+    fn = epi == 1 ? moe_gemm_kernel<1, false>
+                  : (epi == 2 ? moe_gemm_kernel<2, false> : moe_gemm_kernel<3, false>);
+    smem = TileCfg<false>::kSmemBytes;
+  }
+  if (!attr_set[narrow][epi]) {
+    cudaError_t err =
+        cudaFuncSetAttribute((const void*)fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    attr_set[epi] = true;
+    attr_set[narrow][epi] = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

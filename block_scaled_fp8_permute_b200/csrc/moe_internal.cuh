@@ -31,12 +31,15 @@ enum HdrWord : int {
   kHdrSwapExperts = 7,// experts run with swapped operand roles (n <= swap threshold)
   kHdrSwapMax = 8,    // the threshold the plan used
   kHdrPlanDone = 9,   // blocks of the plan's counting kernel that have finished
+  kHdrNarrowMTiles = 10,  // m-tiles of experts run with narrow tiles (1..narrow_max rows)
+  kHdrNarrowMax = 11,     // the narrow threshold the plan used
   kHdrWords = 64
 };
 
 // byte offsets of every region of the workspace (all 1024-byte aligned)
 struct WsLayout {
   size_t hdr, counts, offs, poffs, chunk, row_of, src_of, tile_expert, mpair, norm_mt, swap_e;
+  size_t narrow_mt;
   size_t xp, xp_sf, a2, a2_sf, yp;
   size_t total;
   int R, P_max, MT_max, MP_max, NCH;
@@ -78,6 +81,7 @@ inline WsLayout ws_layout(const moe_shape& s) {
   L.mpair = take((size_t)L.MP_max * 4);
   L.norm_mt = take((size_t)L.MT_max * 4);
   L.swap_e = take((size_t)s.E * 4);
+  L.narrow_mt = take((size_t)s.E * 4);
   L.xp = take((size_t)L.P_max * s.H);
   L.xp_sf = take((size_t)L.MT_max * (s.H / 128) * kSfChunk);
   L.a2 = take((size_t)L.P_max * s.I);
@@ -104,7 +108,8 @@ struct GemmArgs {
   const float* topk_w;     // [T*k]
   int H;
   const int* mpair;        // m-tile pairs: first m-tile | (1 << 31) when the pair has one m-tile
-  const int* norm_mtiles;  // m-tiles of normal-tiled experts
+  const int* norm_mtiles;  // m-tiles this launch runs (normal or narrow list)
+  int tiles_word;          // header word holding their count
   const int* swap_experts; // experts with swapped operand roles
   const int* poffs;        // padded first row of every expert
   const int* counts;       // rows of every expert
@@ -117,6 +122,9 @@ struct GemmArgs {
 
 // experts with at most this many routed rows use swapped operand roles
 constexpr int kMaxSwapRows = 64;
+// narrow tiles: the A operand of a stage holds this many rows (the MMA still
+// spans 128; the rows past them are padding and never stored)
+constexpr int kNarrowRows = 32;
 
 // record the first error of a call in the status word
 __device__ inline void set_status(int* hdr, int code) { atomicCAS(&hdr[kHdrStatus], 0, code); }

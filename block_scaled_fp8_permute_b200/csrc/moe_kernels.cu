@@ -29,13 +29,15 @@ __device__ __forceinline__ size_t sf_chunk_offset(int row, int kg, int G) {
 // block to finish then turns the chunk histograms into per-chunk starting
 // ranks (exclusive, in place), expert counts, offsets, padded offsets, the
 // m-tile -> expert table, the m-tile pairs and m-tiles of normal-tiled
-// experts, the list of swapped-role experts (1 <= count <= swap_max) and -1
+// experts, the list of swapped-role experts (1 <= count <= swap_max), the
+// m-tiles of narrow-tiled experts (1 <= count <= narrow_max) and -1
 // for the padding rows of src_of.
 __global__ void __launch_bounds__(1024) plan_count_scan_kernel(
-    const int32_t* __restrict__ idx, int R, int E, int NCH, int swap_max,
+    const int32_t* __restrict__ idx, int R, int E, int NCH, int swap_max, int narrow_max,
     int* __restrict__ chunk_counts, int* __restrict__ counts, int* __restrict__ offs,
     int* __restrict__ poffs, int* __restrict__ tile_expert, int* __restrict__ mpair,
-    int* __restrict__ norm_mtiles, int* __restrict__ swap_experts, int* __restrict__ src_of,
+    int* __restrict__ norm_mtiles, int* __restrict__ swap_experts, int* __restrict__ narrow_mtiles,
+    int* __restrict__ src_of,
     int* __restrict__ hdr) {
   __shared__ int hist[kMaxE];
   __shared__ int last_block;
@@ -65,11 +67,11 @@ __global__ void __launch_bounds__(1024) plan_count_scan_kernel(
 
   // ---- scan (last block only): count, padded count, m-tile pairs and
   // m-tiles of the normal-tiled experts, swapped-role experts
-  constexpr int NV = 5;
+  constexpr int NV = 6;
   __shared__ int warp_tot[NV][32];
   __shared__ int carry[NV];
   const int lane = tid & 31, wid = tid >> 5;
-  if (tid < 5) carry[tid] = 0;
+  if (tid < NV) carry[tid] = 0;
   __syncthreads();
   for (int e0 = 0; e0 < E; e0 += 1024) {
     const int e = e0 + tid;
@@ -96,11 +98,13 @@ __global__ void __launch_bounds__(1024) plan_count_scan_kernel(
     if (e < E) counts[e] = c;
     const int pc = (c + kBlockM - 1) / kBlockM * kBlockM;
     const bool swapped = c > 0 && c <= swap_max;
-    const int nm = swapped ? 0 : pc / kBlockM;
+    const bool narrow = !swapped && c > 0 && c <= narrow_max;  // one m-tile, <= kNarrowRows rows
+    const int nm = (swapped || narrow) ? 0 : pc / kBlockM;
     const int np = (nm + 1) / 2;
     const int ns = swapped ? 1 : 0;
-    const int val[NV] = {c, pc, np, nm, ns};
-    int incl[NV] = {c, pc, np, nm, ns};
+    const int nn = narrow ? 1 : 0;
+    const int val[NV] = {c, pc, np, nm, ns, nn};
+    int incl[NV] = {c, pc, np, nm, ns, nn};
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
 #pragma unroll
@@ -138,6 +142,7 @@ __global__ void __launch_bounds__(1024) plan_count_scan_kernel(
         mpair[pre[2] + i] = (mt_first + 2 * i) | ((2 * i + 1 == nm) ? (int)0x80000000 : 0);
       for (int i = 0; i < nm; ++i) norm_mtiles[pre[3] + i] = mt_first + i;
       if (swapped) swap_experts[pre[4]] = e;
+      if (narrow) narrow_mtiles[pre[5]] = mt_first;
       for (int r = pre[1] + c; r < pre[1] + pc; ++r) src_of[r] = -1;
     }
     __syncthreads();
@@ -153,6 +158,8 @@ __global__ void __launch_bounds__(1024) plan_count_scan_kernel(
     hdr[kHdrNormMTiles] = carry[3];
     hdr[kHdrSwapExperts] = carry[4];
     hdr[kHdrSwapMax] = swap_max;
+    hdr[kHdrNarrowMTiles] = carry[5];
+    hdr[kHdrNarrowMax] = narrow_max;
   }
 }
 
@@ -384,10 +391,10 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max, int* chunk,
-                        int* counts, int* offs, int* poffs, int* tile_expert, int* mpair,
-                        int* norm_mtiles, int* swap_experts, int* row_of, int* src_of, int* hdr,
-                        bool pdl, cudaStream_t stream) {
+cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max, int narrow_max,
+                        int* chunk, int* counts, int* offs, int* poffs, int* tile_expert,
+                        int* mpair, int* norm_mtiles, int* swap_experts, int* narrow_mtiles,
+                        int* row_of, int* src_of, int* hdr, bool pdl, cudaStream_t stream) {
   static bool attr_set = false;
   const size_t scatter_smem = (size_t)32 * E * sizeof(unsigned short);
   if (!attr_set) {
@@ -398,8 +405,8 @@ cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max,
     attr_set = true;
   }
   plan_count_scan_kernel<<<NCH > 0 ? NCH : 1, 1024, 0, stream>>>(
-      idx, R, E, NCH, swap_max, chunk, counts, offs, poffs, tile_expert, mpair, norm_mtiles,
-      swap_experts, src_of, hdr);
+      idx, R, E, NCH, swap_max, narrow_max, chunk, counts, offs, poffs, tile_expert, mpair,
+      norm_mtiles, swap_experts, narrow_mtiles, src_of, hdr);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || R == 0) return e;
   const int32_t* cidx = idx;

@@ -113,6 +113,16 @@ void moe_set_gemm_variant(int variant);
  * either way.  Process-wide. */
 void moe_set_swap_max(int rows);
 
+/* Narrow tiles for experts with 1..32 routed rows: their A operand stages
+ * only 32 rows per 128-K step, which leaves room for a fifth pipeline stage
+ * and so a deeper stream of the expert's weights (decode-sized batches are
+ * bound by that stream).  -1 (default): on when the layer has at most 128
+ * routed rows per expert on average; 0: off; 1: on.  Never with SM-pair
+ * tiles.  Read by moe_plan and moe_forward, which must see the same value
+ * (set it before moe_plan).  Results are the same either way.
+ * Process-wide. */
+void moe_set_narrow_tiles(int mode);
+
 /* ---------------------------------------------------------------- weights */
 /* Bytes of one transformed weight: which = 1 for W1, 2 for W2.  Returns the
  * FP4 byte count and writes the scale-factor byte count to *sf_bytes (may

@@ -46,18 +46,22 @@ def test_tiny_workload_all_tokens(gemm_variant):
     _check_full(synth.make_inputs(synth.workload("tiny")), "tiny")
 
 
-@pytest.fixture(params=[(0, 64), (0, 0), (1, 64), (1, 0)],
-                ids=["one-sm+swap", "one-sm", "sm-pair+swap", "sm-pair"])
+@pytest.fixture(params=[(0, 64, -1), (0, 0, -1), (0, 0, 1), (0, 0, 0), (1, 64, -1), (1, 0, -1)],
+                ids=["one-sm+swap", "one-sm", "one-sm+narrow", "one-sm-no-narrow",
+                     "sm-pair+swap", "sm-pair"])
 def gemm_variant(request):
     """Tiling of the normal GEMM tiles x the swapped-role threshold (0: every
-    expert uses normal tiles; 64: experts with <= 64 rows use swapped roles)."""
+    expert uses normal tiles; 64: experts with <= 64 rows use swapped roles) x
+    the narrow-tile mode (-1 auto, 1 forced on, 0 off)."""
     import block_scaled_fp8_permute_b200 as moe
-    variant, swap_max = request.param
+    variant, swap_max, narrow = request.param
     moe.moe_set_gemm_variant(variant)
     moe.moe_set_swap_max(swap_max)
+    moe.moe_set_narrow_tiles(narrow)
     yield request.param
     moe.moe_set_gemm_variant(0)
     moe.moe_set_swap_max(0)
+    moe.moe_set_narrow_tiles(-1)
 
 
 @pytest.mark.parametrize("T,H,I,E,k", [
@@ -137,15 +141,18 @@ def _full_inputs(wl):
     return dict(x=x, x_sf=x_sf, topk_idx=idx, topk_w=tw, w1=w1, w1_sf=w1_sf, w2=w2, w2_sf=w2_sf)
 
 
-@pytest.fixture(params=[(0, 0), (0, 64), (1, 0)], ids=["default", "swap", "sm-pair"])
+@pytest.fixture(params=[(0, 0, -1), (0, 0, 0), (0, 64, -1), (1, 0, -1)],
+                ids=["default", "no-narrow", "swap", "sm-pair"])
 def full_variant(request):
     import block_scaled_fp8_permute_b200 as moe
-    variant, swap_max = request.param
+    variant, swap_max, narrow = request.param
     moe.moe_set_gemm_variant(variant)
     moe.moe_set_swap_max(swap_max)
+    moe.moe_set_narrow_tiles(narrow)
     yield request.param
     moe.moe_set_gemm_variant(0)
     moe.moe_set_swap_max(0)
+    moe.moe_set_narrow_tiles(-1)
 
 
 @pytest.mark.parametrize("name,n_sample", [
