@@ -394,7 +394,10 @@ def run_ours(args, wl, dist, rank, world, local_rank):
                           "algorithmic_bytes": step_bytes, "experts_touched": touched},
         "e2e": {"value": flops / (e2e * 1e-3) / 1e12, "unit": "TFLOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
-        "gpu_launches": 6 * K,  # count+scan, scatter, permute, linear1, linear2, combine
+        # count+scan, scatter, permute, linear1, linear2, combine; with narrow tiles (the
+        # library's default when the layer has <= 128 rows per expert) a second linear1
+        # and linear2 launch run the narrow m-tiles
+        "gpu_launches": (6 + (2 if wl.R <= 128 * wl.E else 0)) * K,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
     }
