@@ -121,6 +121,10 @@ class ClockSampler:
                     return
                 time.sleep(0.0002)
 
+        # the launching thread holds the GIL while it enqueues the steps: switch
+        # threads often, or a short timed region gets a single sample
+        self.switch = sys.getswitchinterval()
+        sys.setswitchinterval(0.0001)
         self.thread = threading.Thread(target=loop, daemon=True)
         self.thread.start()
         return self
@@ -129,6 +133,7 @@ class ClockSampler:
         if self.nv is not None:
             self.stop.set()
             self.thread.join(timeout=5)
+            sys.setswitchinterval(self.switch)
 
     def summary(self):
         out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
