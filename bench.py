@@ -144,14 +144,34 @@ class ClockSampler:
         return out
 
 
-def _dist():
+def _dist(backend="nccl"):
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws == 1:
         return None, 0, 1, 0
     import torch.distributed as dist
     from datetime import timedelta
-    dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dist.init_process_group(backend, timeout=timedelta(seconds=120))
     return dist, dist.get_rank(), ws, int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def replica_inputs(wl, rank):
+    """Inputs of one replica: the weights are the workload's (shared by every
+    rank), the activations and routing are seeded by seed + rank."""
+    import synth
+    wl_r = wl if rank == 0 else synth.Workload(**{**wl.__dict__, "seed": wl.seed + rank})
+    x, x_sf, idx, tw = synth.make_activations(wl_r)
+    w1, w1_sf, w2, w2_sf = synth.make_weights(wl)
+    return dict(x=x, x_sf=x_sf, topk_idx=idx, topk_w=tw, w1=w1, w1_sf=w1_sf, w2=w2, w2_sf=w2_sf)
+
+
+def max_over_ranks(v, dist, device):
+    """The largest of every rank's v (one all-reduce; the value itself at N = 1)."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def _workload_desc(wl):
@@ -232,16 +252,11 @@ def run_ours(args, wl, dist, rank, world, local_rank):
     import torch
 
     import block_scaled_fp8_permute_b200 as moe
-    import synth
     from tests.gpu_util import Layer
 
     torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
-    # each replica: shared weights, its own activations / routing
-    wl_r = wl if rank == 0 else synth.Workload(**{**wl.__dict__, "seed": wl.seed + rank})
-    x, x_sf, idx, tw = synth.make_activations(wl_r)
-    w1, w1_sf, w2, w2_sf = synth.make_weights(wl)
-    inputs = dict(x=x, x_sf=x_sf, topk_idx=idx, topk_w=tw, w1=w1, w1_sf=w1_sf, w2=w2, w2_sf=w2_sf)
+    inputs = replica_inputs(wl, rank)  # shared weights, this replica's activations / routing
     lay = Layer(inputs, device=dev)
     shp, d = lay.shape, lay.dev
     stream = torch.cuda.current_stream()
@@ -331,16 +346,9 @@ def run_ours(args, wl, dist, rank, world, local_rank):
             e2e_ms.append(e0.elapsed_time(e1))
     e2e = statistics.mean(e2e_ms)
 
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    ms = max_over_ranks(ms)
-    e2e = max_over_ranks(e2e)
-    g1 = max_over_ranks(kern["linear1"])
+    ms = max_over_ranks(ms, dist, dev)
+    e2e = max_over_ranks(e2e, dist, dev)
+    g1 = max_over_ranks(kern["linear1"], dist, dev)
     if rank != 0:
         return
     flops = wl.flops * world
