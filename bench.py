@@ -76,14 +76,16 @@ def _peaks():
 
 class ClockSampler:
     """SM clock and clock-event reasons sampled through NVML every ~0.2 ms in a
-    background thread while the timed region runs."""
+    background thread.  mark("start") / mark("end") bracket the timed region;
+    the sampler may keep running over later steps of the same workload, which
+    summary() reports separately."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
 
     def __init__(self, cuda_index: int):
         self.cuda_index = cuda_index
-        self.samples, self.reasons, self.max_mhz, self.err = [], set(), None, None
+        self.samples, self.max_mhz, self.err, self.marks = [], None, None, {}
 
     def _handle(self, nv):
         import torch
@@ -94,6 +96,9 @@ class ClockSampler:
             return nv.nvmlDeviceGetHandleByUUID(uuid.encode())
         except Exception:
             return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
+
+    def mark(self, name):
+        self.marks[name] = time.perf_counter()
 
     def __enter__(self):
         import threading
@@ -110,12 +115,9 @@ class ClockSampler:
         def loop():
             while not self.stop.is_set():
                 try:
-                    self.samples.append(float(self.nv.nvmlDeviceGetClockInfo(self.h,
-                                                                             self.nv.NVML_CLOCK_SM)))
+                    mhz = float(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
                     bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                    for name, bit in self.REASONS.items():
-                        if bits & bit:
-                            self.reasons.add(name)
+                    self.samples.append((time.perf_counter(), mhz, bits))
                 except Exception as e:
                     self.err = str(e)
                     return
@@ -135,10 +137,19 @@ class ClockSampler:
             self.thread.join(timeout=5)
             sys.setswitchinterval(self.switch)
 
+    def _stats(self, rows):
+        reasons = sorted({n for _, _, bits in rows for n, bit in self.REASONS.items() if bits & bit})
+        return (statistics.median([m for _, m, _ in rows]) if rows else None), reasons, len(rows)
+
     def summary(self):
-        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-               "samples": len(self.samples)}
+        t0, t1 = self.marks.get("start", float("-inf")), self.marks.get("end", float("inf"))
+        timed = [r for r in self.samples if t0 <= r[0] <= t1]
+        mhz, reasons, n = self._stats(timed)
+        out = {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": n}
+        if len(self.samples) > len(timed):
+            mhz_all, reasons_all, n_all = self._stats(self.samples)
+            out["with_following_steps"] = {"sm_mhz": mhz_all, "reasons": reasons_all,
+                                           "samples": n_all}
         if self.err:
             out["note"] = self.err
         return out
@@ -293,13 +304,23 @@ def run_ours(args, wl, dist, rank, world, local_rank):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        for i in range(K):
-            flush.zero_()
-            ev[i][0].record(stream)
-            graph.replay()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    for row in kev:
+        for e in row:
+            e.record(stream)  # materialise the handles
+    torch.cuda.synchronize()
+    # clocks: sampled over the timed region (marked) and, as more evidence for a short
+    # region, over the eager kernel-timing steps that follow it
+    clk = ClockSampler(local_rank)
+    clk.__enter__()
+    clk.mark("start")
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        graph.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clk.mark("end")
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -307,11 +328,6 @@ def run_ours(args, wl, dist, rank, world, local_rank):
 
     # Kernel durations: the same steps run eagerly with events at the kernel
     # boundaries (moe_set_timing_events), K more steps.
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
-    for row in kev:
-        for e in row:
-            e.record(stream)  # materialise the handles
-    torch.cuda.synchronize()
     for i in range(K):
         flush.zero_()
         kev[i][0].record(stream)
@@ -319,6 +335,7 @@ def run_ours(args, wl, dist, rank, world, local_rank):
         step()
     moe.moe_set_timing_events(None)
     torch.cuda.synchronize()
+    clk.__exit__(None, None, None)
     kern = {name: statistics.mean(kev[i][a].elapsed_time(kev[i][b]) for i in range(K))
             for name, a, b in (("plan", 0, 1), ("permute", 1, 2), ("linear1", 2, 3),
                                ("linear2", 3, 4), ("combine", 4, 5))}
@@ -471,12 +488,14 @@ def run_gemm(args, name):
     K_ = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
     with ClockSampler(0) as clk:
+        clk.mark("start")
         for i in range(K_):
             flush.zero_()
             ev[i][0].record(stream)
             graph.replay()
             ev[i][1].record(stream)
         torch.cuda.synchronize()
+        clk.mark("end")
     ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K_))
     rows = int(counts.sum())
     flops = 2.0 * rows * N * K
