@@ -100,6 +100,13 @@ class ClockSampler:
     def mark(self, name):
         self.marks[name] = time.perf_counter()
 
+    def wait_first(self, timeout=1.0):
+        """Block until the sampling thread has taken its first sample (its start-up
+        and NVML's first call would otherwise eat a short timed region)."""
+        t_end = time.perf_counter() + timeout
+        while self.nv is not None and not self.samples and time.perf_counter() < t_end:
+            time.sleep(0.0005)
+
     def __enter__(self):
         import threading
         try:
@@ -313,6 +320,7 @@ def run_ours(args, wl, dist, rank, world, local_rank):
     # region, over the eager kernel-timing steps that follow it
     clk = ClockSampler(local_rank)
     clk.__enter__()
+    clk.wait_first()
     clk.mark("start")
     for i in range(K):
         flush.zero_()
@@ -488,6 +496,7 @@ def run_gemm(args, name):
     K_ = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_)]
     with ClockSampler(0) as clk:
+        clk.wait_first()
         clk.mark("start")
         for i in range(K_):
             flush.zero_()
