@@ -16,7 +16,7 @@
 //   warp 0     TMA producer: A tile 128x128 (E4M3), B tile 256x128 (E2M1,
 //              unpacked by the TMA to one byte per element as the block-scaled
 //              MMA requires), and the two 512/1024-byte scale chunks, into a
-//              4-stage shared-memory ring.
+//              shared-memory ring (4 stages; 5 for narrow tiles, TileCfg).
 //   warp 1     TMEM allocator and MMA issuer: copies the stage's scales into
 //              TMEM (tcgen05.cp) and issues 4 x tcgen05.mma kind::mxf8f6f4
 //              (M=128, N=256, K=32) per stage into one FP32 TMEM accumulator.

@@ -242,7 +242,8 @@ moe_status moe_plan_export(const moe_shape* shape, const void* workspace, int32_
 /* Kernel timing: when `events` is not NULL and n >= 5, every following
  * moe_forward records events[0..4] (cudaEvent_t handles owned by the
  * caller) on its stream: before the permute kernel, after it, after the
- * linear1 kernel, after the linear2 kernel and after the combine kernel.
+ * linear1 kernels, after the linear2 kernels (normal, narrow and swapped-role
+ * tiles each) and after the combine kernel.
  * NULL stops it.  Process-wide; the handles must outlive their use. */
 void moe_set_timing_events(void* const* events, int n);
 
