@@ -64,6 +64,9 @@ WORKLOADS = {
     "usage": Workload("usage", 8192, 7168, 8, 2, 9216, 0, 0.0),
     "skewed": Workload("skewed", 4096, 7168, 256, 8, 2048, 1, 1.1),
     "decode": Workload("decode", 128, 7168, 256, 8, 2048, 1, 0.0),
+    # a profiling-sized decode layer: the decode shape with 64 experts (1.4 GB of
+    # FP4 weights, still far above L2), small enough for a multi-pass ncu capture
+    "decode-e64": Workload("decode-e64", 128, 7168, 64, 8, 2048, 1, 0.0),
 }
 
 
