@@ -172,12 +172,13 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 // (experts with 1..kNarrowRows rows) with one-SM tiles when the layer has at
 // most 128 rows per expert on average (decode-sized and fine-grained layers),
 // or always / never when set so; off with SM-pair tiles.
-int narrow_max_for(const moe_shape& s) {
-  if (g_gemm_variant.load() == 1) return 0;
+bool narrow_enabled(const moe_shape& s) {
   const int mode = g_narrow_mode.load();
-  if (mode == 0) return 0;
-  if (mode < 0 && (long long)s.T * s.topk > (long long)kBlockM * s.E) return 0;
-  return kNarrowRows;
+  if (mode == 0) return false;
+  return mode > 0 || (long long)s.T * s.topk <= (long long)kBlockM * s.E;
+}
+int narrow_max_for(const moe_shape& s) {
+  return (g_gemm_variant.load() != 1 && narrow_enabled(s)) ? kNarrowRows : 0;
 }
 
 // standalone GEMM: shape rules and workspace (header, tile lists, A's scale chunks)
@@ -412,7 +413,9 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   const bool pair1 = g_gemm_variant.load() == 1;
   const bool pair2 = pair1 && (sh.H % 256) == 0;
   CUtensorMap tmX, tmW1, tmA2, tmW2, tmYp, tmXsf, tmW1sf, tmA2sf, tmW2sf;
-  CUtensorMap tmX16, tmA216, tmW1s, tmW2s;  // swapped-role kernel: 16-row token boxes
+  // swapped-role kernel: 16-row token boxes; tmW1s / tmW2s (256-row weight boxes)
+  // also serve the narrow tiles
+  CUtensorMap tmX16, tmA216, tmW1s, tmW2s;
   CUtensorMap tmXn, tmA2n;                   // narrow tiles: kNarrowRows-row A boxes
   if (!encode_act(&tmXn, ws.xp(), ws.L.P_max, sh.H, kNarrowRows) ||
       !encode_act(&tmA2n, ws.a2(), ws.L.P_max, sh.I, kNarrowRows))
@@ -473,14 +476,17 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
     e = launch_gemm(1, false, tmX, tmW1, tmYp, g1, grid1 < 1 ? 1 : grid1, pdl, s);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  // experts with at most kNarrowRows rows: narrow tiles (a deeper weight stream)
-  const bool narrow = narrow_max_for(sh) > 0;
+  // experts with at most kNarrowRows rows: narrow tiles (a deeper weight stream).
+  // Launched whenever the plan may have listed such experts, also if the tiling
+  // variant was switched after the plan (an empty list costs one short launch).
+  const bool narrow = narrow_enabled(sh);
   const int narrow_grid1 = (int)((long long)sh.E * NT1 < sms ? (long long)sh.E * NT1 : sms);
   if (narrow) {
     GemmArgs g1n = g1;
     g1n.norm_mtiles = ws.narrow_mt();
     g1n.tiles_word = kHdrNarrowMTiles;
-    e = launch_gemm(1, true, tmXn, tmW1, tmYp, g1n, narrow_grid1, pdl, s);
+    // 256-row weight boxes, whatever box the SM-pair tiles use
+    e = launch_gemm(1, true, tmXn, tmW1s, tmYp, g1n, narrow_grid1, pdl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
   // swapped-role tiles exist only when the plan was made with a threshold > 0
@@ -515,7 +521,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
     g2n.norm_mtiles = ws.narrow_mt();
     g2n.tiles_word = kHdrNarrowMTiles;
     const int narrow_grid2 = (int)((long long)sh.E * NT2 < sms ? (long long)sh.E * NT2 : sms);
-    e = launch_gemm(2, true, tmA2n, tmW2, tmYp, g2n, narrow_grid2, pdl, s);
+    e = launch_gemm(2, true, tmA2n, tmW2s, tmYp, g2n, narrow_grid2, pdl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
   if (use_swap) {

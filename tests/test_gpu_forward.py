@@ -89,6 +89,28 @@ def test_unused_slots_duplicates_and_bad_ids(gemm_variant):
     assert lay.status() == 6
 
 
+@pytest.mark.parametrize("plan_variant,fwd_variant", [(0, 1), (1, 0)])
+def test_tiling_switched_between_plan_and_forward(plan_variant, fwd_variant):
+    """Many small experts (narrow tiles with one-SM tiling): the plan made with
+    one tiling variant, the forward run with the other, still computes every row."""
+    import block_scaled_fp8_permute_b200 as moe
+    d = _inputs(200, 512, 128, 64, 6, seed=4)
+    try:
+        moe.moe_set_gemm_variant(plan_variant)
+        lay = Layer(d)
+        moe.moe_plan(lay.shape, lay.dev["topk_idx"], lay.ws)
+        moe.moe_set_gemm_variant(fwd_variant)
+        dv = lay.dev
+        moe.moe_forward(lay.shape, dv["x"], dv["x_sf"], dv["topk_idx"], dv["topk_w"], *lay.wt,
+                        lay.y, lay.ws)
+        y = lay.y_bits()
+    finally:
+        moe.moe_set_gemm_variant(0)
+    y_ref, _, _ = oracle.moe_forward(**d)
+    assert_parity(y, y_ref, f"plan {plan_variant} forward {fwd_variant}")
+    assert lay.status() == 0
+
+
 def test_all_rows_one_expert_and_empty_experts():
     d = _inputs(200, 256, 256, 8, 2, seed=9)
     d["topk_idx"][:, 0] = 3
