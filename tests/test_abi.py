@@ -134,3 +134,27 @@ def test_gemm_sizes_and_validation(moe):
     # no rows: nothing to do
     ws0 = moe.moe_gemm_workspace_bytes(1, 0, 256, 512)
     assert lib.moe_gemm_fp8_fp4(0, 256, 512, None, None, None, None, None, 4096, ws0, None) == 0
+
+
+def test_product_path_never_touches_the_oracle():
+    """The library package and its CUDA sources name nothing under oracle/."""
+    pkg = os.path.join(ROOT, "block_scaled_fp8_permute_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"\boracle\b", src), f
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """No CPU fallback: importing the binding where libmoe.so is absent raises."""
+    import importlib.util
+    import shutil
+    pkg = tmp_path / "moe_pkg_copy"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "block_scaled_fp8_permute_b200", "__init__.py"),
+                pkg / "__init__.py")
+    spec = importlib.util.spec_from_file_location("moe_pkg_copy", pkg / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)
