@@ -30,10 +30,12 @@
  *   - the SwiGLU output is rounded to float, then requantised to E4M3
  *     (round to nearest even, saturating) with the rule above; linear2
  *     consumes the decoded requantised values.
- *   - the top-k weight multiplies the linear2 output of its slot and the
- *     product is rounded to BF16 (the FP8 x FP4 GEMM emits BF16 output,
- *     [EXPLAINER] 4.3); the BF16 slot values are summed in slot order in
- *     double; y = BF16 round-to-nearest-even of that sum.
+ *   - the top-k weight multiplies the linear2 output of its slot; the
+ *     weighted outputs are summed in slot order in double and y is the one
+ *     BF16 round-to-nearest-even of that sum.  The fused operator keeps the
+ *     expert outputs on chip up to the combine ([EXPLAINER] 3.2), so no
+ *     intermediate rounding other than the FP8 requantisation of the
+ *     SwiGLU output is part of the definition.
  *   - topk_idx == -1 means "slot unused"; any other id outside [0, E) is
  *     counted as invalid and skipped.
  *   - rows of one expert are ordered by ascending flattened index t*k+s.
@@ -209,14 +211,6 @@ int orc_plan(int T, int k, int E, int bm, const int32_t* topk_idx, int32_t* coun
   return bad;
 }
 
-/* BF16 bit pattern -> value (the upper half of an IEEE binary32). */
-static double bf16_value(uint16_t b) {
-  uint32_t bits = (uint32_t)b << 16;
-  float f;
-  memcpy(&f, &bits, 4);
-  return (double)f;
-}
-
 /* ------------------------------------------------------------------------ */
 /* The layer forward ([EXPLAINER] 3.1 and 3.3; [OVERVIEW] 5).               */
 /* ------------------------------------------------------------------------ */
@@ -230,7 +224,7 @@ static double bf16_value(uint16_t b) {
  *   w2     u8  [E, H, I/2],  w2_sf u8 [E, H, I/32]
  * Computes y for the tokens in token_list (n_list of them) into
  * y_out [n_list, H] (bf16 bits) and, when acc_out is not NULL, the double
- * sum of the BF16 slot values before the final rounding [n_list, H].
+ * sum of the weighted slot outputs before the final rounding [n_list, H].
  * Returns the number of invalid expert ids met. */
 
 static inline double x_value(const uint8_t* x, const int32_t* x_sf, int H, int t, int h) {
@@ -287,13 +281,12 @@ int orc_moe_forward(int T, int H, int I, int E, int k, const uint8_t* x, const i
         orc_requant_block(af + 32 * b, 32, q + 32 * b, &sb);
         for (int j = 32 * b; j < 32 * b + 32; ++j) ad[j] = orc_e4m3_value(q[j]) * orc_ue8m0_value(sb);
       }
-      /* linear2, weighted and rounded to BF16, then combined:
-       * acc[n] += bf16(w * sum_j a[j] * W2[e][n][j]) */
+      /* linear2, weighted, combined in double: acc[n] += w * sum_j a[j] * W2[e][n][j] */
       double wt = (double)topk_w[(size_t)t * k + s];
       for (int n = 0; n < H; ++n) {
         double sum = 0.0;
         for (int j = 0; j < I; ++j) sum += ad[j] * w_value(w2, w2_sf, H, I, e, n, j);
-        acc[n] += bf16_value(orc_bf16_rne(wt * sum));
+        acc[n] += wt * sum;
       }
     }
     for (int n = 0; n < H; ++n) {

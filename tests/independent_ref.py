@@ -106,7 +106,7 @@ def bf16_value(v: np.ndarray) -> np.ndarray:
 
 def moe_masked(x, x_sf, topk_idx, topk_w, w1, w1_sf, w2, w2_sf):
     """Masked all-experts formulation:
-    acc[t] = sum_e sum_s [idx[t,s]==e] bf16(w[t,s] FFN_e(x_t)).
+    acc[t] = sum_e sum_s [idx[t,s]==e] w[t,s] FFN_e(x_t).
 
     Returns the float64 accumulator [T, H]."""
     T, H = x.shape
@@ -124,5 +124,5 @@ def moe_masked(x, x_sf, topk_idx, topk_w, w1, w1_sf, w2, w2_sf):
         O = ad @ W2[e].T                                  # [T, H]
         for s in range(topk_idx.shape[1]):
             sel = (topk_idx[:, s] == e).astype(np.float64) * topk_w[:, s].astype(np.float64)
-            acc += bf16_value(sel[:, None] * O)
+            acc += sel[:, None] * O
     return acc

@@ -141,7 +141,7 @@ def test_dense_ffn_special_case():
     G = X @ W1.T
     a = (G[:, :128] / (1 + np.exp(-G[:, :128])) * G[:, 128:]).astype(np.float32)
     ad, _, _ = ind.requant(a)
-    ref = ind.bf16_value(ad @ W2.T)  # the GEMM's BF16 output, weight 1
+    ref = ad @ W2.T  # weight 1: the accumulator is the FFN output itself
     np.testing.assert_allclose(acc, ref, rtol=1e-11, atol=1e-12 * np.abs(ref).max())
 
 
@@ -151,6 +151,8 @@ def test_masked_all_experts_brute_force(T, E, k):
     y, acc, _ = oracle.moe_forward(**d, want_acc=True)
     ref = ind.moe_masked(**d)
     np.testing.assert_allclose(acc, ref, rtol=1e-11, atol=1e-12 * np.abs(ref).max())
+    # y is the one BF16 rounding of that double sum (no per-slot rounding before it)
+    assert np.array_equal(oracle.bf16_bits_to_float(y).astype(np.float64), ind.bf16_value(ref))
 
 
 # ------------------------------------------------------------- invariants
