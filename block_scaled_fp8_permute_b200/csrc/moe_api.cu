@@ -41,6 +41,17 @@ std::atomic<int> g_pdl{1};
 std::atomic<int> g_gemm_variant{0};
 std::atomic<int> g_swap_max{0};
 std::atomic<int> g_narrow_mode{-1};
+// Every value the two plan-time knobs have held in this process.  moe_plan
+// takes the knobs' values at plan time and moves the experts it gives to
+// narrow or swapped-role tiles out of the normal tile list; moe_forward
+// launches those kernels whenever any value seen so far could have listed
+// such experts, so changing a knob between moe_plan and moe_forward (or from
+// another thread) never drops rows.  The launched kernels read the plan's
+// own counts on the device and exit at once when their list is empty.
+std::atomic<int> g_narrow_modes_seen{1};  // bit 0: auto (-1), bit 1: off (0), bit 2: on (1)
+std::atomic<int> g_swap_max_seen{0};      // largest swapped-role threshold ever set
+std::atomic<int> g_fault_skip_it{0};               // test hook, 0 = off
+std::atomic<unsigned long long> g_fault_wait_ns{0}; // test hook, 0 = default limits
 std::mutex g_ev_mu;
 cudaEvent_t g_events[5];
 bool g_events_on = false;
@@ -172,13 +183,22 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 // (experts with 1..kNarrowRows rows) with one-SM tiles when the layer has at
 // most 128 rows per expert on average (decode-sized and fine-grained layers),
 // or always / never when set so; off with SM-pair tiles.
+bool narrow_auto_on(const moe_shape& s) {
+  return (long long)s.T * s.topk <= (long long)kBlockM * s.E;
+}
 bool narrow_enabled(const moe_shape& s) {
   const int mode = g_narrow_mode.load();
   if (mode == 0) return false;
-  return mode > 0 || (long long)s.T * s.topk <= (long long)kBlockM * s.E;
+  return mode > 0 || narrow_auto_on(s);
 }
 int narrow_max_for(const moe_shape& s) {
   return (g_gemm_variant.load() != 1 && narrow_enabled(s)) ? kNarrowRows : 0;
+}
+// Could a plan of this shape made at any time in this process have listed
+// narrow-tiled experts?  (A superset of the plan's actual choice.)
+bool narrow_possible(const moe_shape& s) {
+  const int seen = g_narrow_modes_seen.load();
+  return (seen & 4) != 0 || ((seen & 1) != 0 && narrow_auto_on(s));
 }
 
 // standalone GEMM: shape rules and workspace (header, tile lists, A's scale chunks)
@@ -310,10 +330,18 @@ void moe_set_pdl(int enable) { g_pdl.store(enable ? 1 : 0); }
 
 void moe_set_gemm_variant(int variant) { g_gemm_variant.store(variant == 1 ? 1 : 0); }
 
-void moe_set_narrow_tiles(int mode) { g_narrow_mode.store(mode < 0 ? -1 : (mode ? 1 : 0)); }
+void moe_set_narrow_tiles(int mode) {
+  const int m = mode < 0 ? -1 : (mode ? 1 : 0);
+  g_narrow_modes_seen.fetch_or(m < 0 ? 1 : (m == 0 ? 2 : 4));  // before any plan can use it
+  g_narrow_mode.store(m);
+}
 
 void moe_set_swap_max(int rows) {
-  g_swap_max.store(rows < 0 ? 0 : (rows > kMaxSwapRows ? kMaxSwapRows : rows));
+  const int r = rows < 0 ? 0 : (rows > kMaxSwapRows ? kMaxSwapRows : rows);
+  int seen = g_swap_max_seen.load();
+  while (r > seen && !g_swap_max_seen.compare_exchange_weak(seen, r)) {
+  }
+  g_swap_max.store(r);
 }
 
 void moe_set_timing_events(void* const* events, int n) {
@@ -466,6 +494,9 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   g1.a2_sf = ws.a2_sf();
   g1.I = sh.I;
   g1.H = sh.H;
+  GemmArgs g1f = g1;  // the normal one-SM linear1 launch carries the test hook
+  g1f.fault_skip_it = g_fault_skip_it.load();
+  g1f.wait_limit_ns = g_fault_wait_ns.load();
   if (pair1) {
     long long work = (long long)ws.L.MP_max * NT1;
     int pairs = (int)(work < max_pairs_grid ? work : max_pairs_grid);
@@ -473,13 +504,13 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   } else {
     long long tiles1 = (long long)ws.L.MT_max * NT1;
     int grid1 = (int)(tiles1 < sms ? tiles1 : sms);
-    e = launch_gemm(1, false, tmX, tmW1, tmYp, g1, grid1 < 1 ? 1 : grid1, pdl, s);
+    e = launch_gemm(1, false, tmX, tmW1, tmYp, g1f, grid1 < 1 ? 1 : grid1, pdl, s);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   // experts with at most kNarrowRows rows: narrow tiles (a deeper weight stream).
-  // Launched whenever the plan may have listed such experts, also if the tiling
-  // variant was switched after the plan (an empty list costs one short launch).
-  const bool narrow = narrow_enabled(sh);
+  // Launched whenever the plan may have listed such experts, whatever the knobs
+  // say now (an empty list costs one short launch).
+  const bool narrow = narrow_possible(sh);
   const int narrow_grid1 = (int)((long long)sh.E * NT1 < sms ? (long long)sh.E * NT1 : sms);
   if (narrow) {
     GemmArgs g1n = g1;
@@ -490,7 +521,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
   // swapped-role tiles exist only when the plan was made with a threshold > 0
-  const bool use_swap = g_swap_max.load() > 0;
+  const bool use_swap = g_swap_max_seen.load() > 0;
   if (use_swap) {
     const int swap_grid1 = (int)((long long)sh.E * NT1 < sms ? (long long)sh.E * NT1 : sms);
     e = launch_gemm_swap(1, tmW1s, tmX16, g1, swap_grid1, pdl, s);
@@ -577,6 +608,20 @@ moe_status moe_forward_host(const moe_shape* shape, const uint8_t* x_host,
   e = cudaMemcpyAsync(y_host, base + hs.y, ny, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   return cuda_status(e);
+}
+
+void moe_debug_set_fault(int skip_iteration, unsigned long long wait_limit_ns) {
+  g_fault_skip_it.store(skip_iteration >= 0 ? skip_iteration + 1 : 0);
+  g_fault_wait_ns.store(wait_limit_ns);
+}
+
+int moe_get_timeout_site(const void* workspace, moe_stream_t stream) {
+  if (!workspace) return -1;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return -1;
+  int hdr[kHdrWords];
+  if (cudaMemcpy(hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
+  return hdr[kHdrTimeoutSite];
 }
 
 moe_status moe_get_device_status(const void* workspace, moe_stream_t stream) {

@@ -111,6 +111,32 @@ def test_tiling_switched_between_plan_and_forward(plan_variant, fwd_variant):
     assert lay.status() == 0
 
 
+@pytest.mark.parametrize("knob,plan_value,fwd_value", [
+    ("narrow", 1, 0), ("narrow", 0, 1), ("narrow", -1, 0), ("swap", 64, 0), ("swap", 0, 64)])
+def test_knob_changed_between_plan_and_forward(knob, plan_value, fwd_value):
+    """The plan moves small experts to narrow or swapped-role tiles according
+    to the knobs' values at plan time; changing a knob before the forward must
+    not drop those experts' rows (status stays 0, y matches the oracle)."""
+    import block_scaled_fp8_permute_b200 as moe
+    d = _inputs(200, 512, 128, 64, 6, seed=11)   # ~19 rows per expert
+    setter = moe.moe_set_narrow_tiles if knob == "narrow" else moe.moe_set_swap_max
+    default = -1 if knob == "narrow" else 0
+    try:
+        setter(plan_value)
+        lay = Layer(d)
+        moe.moe_plan(lay.shape, lay.dev["topk_idx"], lay.ws)
+        setter(fwd_value)
+        dv = lay.dev
+        moe.moe_forward(lay.shape, dv["x"], dv["x_sf"], dv["topk_idx"], dv["topk_w"], *lay.wt,
+                        lay.y, lay.ws)
+        y = lay.y_bits()
+    finally:
+        setter(default)
+    y_ref, _, _ = oracle.moe_forward(**d)
+    assert_parity(y, y_ref, f"{knob} {plan_value} -> {fwd_value}")
+    assert lay.status() == 0
+
+
 def test_all_rows_one_expert_and_empty_experts():
     d = _inputs(200, 256, 256, 8, 2, seed=9)
     d["topk_idx"][:, 0] = 3
