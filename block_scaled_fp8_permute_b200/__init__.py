@@ -60,6 +60,8 @@ _SIGS = {
     "moe_workspace_bytes_host": (_sz, [_shp]),
     "moe_forward_host": (_i, [_shp] + [_vp] * 9 + [_vp, _sz, _vp]),
     "moe_get_device_status": (_i, [_vp, _vp]),
+    "moe_get_timeout_site": (_i, [_vp, _vp]),
+    "moe_debug_set_fault": (None, [_i, ctypes.c_ulonglong]),
     "moe_plan_max_rows": (_i, [_shp]),
     "moe_plan_export": (_i, [_shp, _vp] + [_vp] * 6 + [_vp]),
     "moe_debug_requant": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
@@ -200,6 +202,14 @@ def moe_forward_noalloc(shp, x, x_sf, topk_idx, topk_w, w1_t, w1_sf_t, w2_t, w2_
 
 def moe_get_device_status(workspace, stream=None) -> int:
     return _lib.moe_get_device_status(_ptr(workspace), _stream(stream))
+
+
+def moe_get_timeout_site(workspace, stream=None) -> int:
+    return _lib.moe_get_timeout_site(_ptr(workspace), _stream(stream))
+
+
+def moe_debug_set_fault(skip_iteration: int, wait_limit_ns: int = 0) -> None:
+    _lib.moe_debug_set_fault(int(skip_iteration), int(wait_limit_ns))
 
 
 def moe_plan_max_rows(shp: MoeShape) -> int:

@@ -132,13 +132,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   pdl_wait();  // inputs come from the previous kernel of the forward
   const int NT = args.NT, KB = args.KB, n_rows = args.n_rows;
+  // wait limits: a stage's data (MMA issuer) gets L, the waits that can only
+  // end after such a stage (free slots, the accumulator) get 2L, so that the
+  // wait nearest the cause expires first
+  const unsigned long long lim = args.wait_limit_ns ? args.wait_limit_ns : kWaitLimitNs;
   const int num_tiles = args.hdr[args.tiles_word] * NT;
 
+  // stages the producer has issued loads into, and the phase of the last one
+  // (producer lane only): after a failure they are waited for before exit
+  uint32_t issued_mask = 0, last_phase = 0;
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t it = 0;
-      uint32_t issued_mask = 0, last_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int mt = args.norm_mtiles[tile / NT], nt = tile - (tile / NT) * NT;
@@ -151,13 +157,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
-          if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
-            set_status(args.hdr, MOE_ERR_TIMEOUT);
-            args.hdr[kHdrTimeoutSite] = 10 + kEpi;
+          if (!mbar_wait_or_abort(&empty[s], ph ^ 1, 2 * lim, abort_flag)) {
+            if (!*abort_flag) record_timeout(args.hdr, 10 + kEpi);
             *abort_flag = 1;
             ok = false;
             break;
           }
+          if ((int)it + 1 == args.fault_skip_it) continue;  // test hook: this stage never fills
           mbar_arrive_expect_tx(&full[s], tx);
           tma_load_2d(sA + s * kSmemA, &tmA, &full[s], kb * kBlockK, mt * kBlockM);
           tma_load_3d(sB + s * kSmemB, &tmB, &full[s], 0, n0, e * KB + kb);
@@ -167,11 +173,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           issued_mask |= 1u << s;
           last_phase = (last_phase & ~(1u << s)) | (ph << s);
         }
-      }
-      if (!ok) {
-        // let copies already in flight land before the CTA's memory goes away
-        for (int s = 0; s < kStages; ++s)
-          if (issued_mask & (1u << s)) (void)mbar_wait(&full[s], (last_phase >> s) & 1);
       }
     }
   } else if (warp == 1) {
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int nt = tile % NT;
         const int n_tile = min(kBlockN, n_rows - nt * kBlockN);
         const uint32_t idesc0 = idesc_mxf8f6f4(/*A E4M3*/ 0, /*B E2M1*/ 5, kBlockM, n_tile);
-        if (!mbar_wait(acc_empty, (ti & 1) ^ 1) || *abort_flag) {
+        if (!mbar_wait_or_abort(acc_empty, (ti & 1) ^ 1, 2 * lim, abort_flag)) {
           ok = false;
           break;
         }
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
-          if (!mbar_wait(&full[s], ph) || *abort_flag) {
+          if (!mbar_wait_or_abort(&full[s], ph, lim, abort_flag)) {
             ok = false;
             break;
           }
@@ -219,8 +220,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_commit(acc_full);
       }
       if (!ok) {
-        set_status(args.hdr, MOE_ERR_TIMEOUT);
-        args.hdr[kHdrTimeoutSite] = 20 + kEpi;
+        if (!*abort_flag) record_timeout(args.hdr, 20 + kEpi);
         *abort_flag = 1;
         if (issued_any) {  // wait for the MMAs in flight before TMEM is released
           tc_commit(drain);
@@ -239,11 +239,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++ti) {
       const int mt = args.norm_mtiles[tile / NT], nt = tile - (tile / NT) * NT;
       // warp-uniform decision: every lane leaves or every lane continues
-      const bool ready = __all_sync(0xffffffffu, mbar_wait(acc_full, ti & 1) && !*abort_flag);
+      const bool ready =
+          __all_sync(0xffffffffu, mbar_wait_or_abort(acc_full, ti & 1, 2 * lim, abort_flag));
       if (!ready) {
         if (lane == 0) {
-          set_status(args.hdr, MOE_ERR_TIMEOUT);
-          args.hdr[kHdrTimeoutSite] = 30 + kEpi;
+          if (!*abort_flag) record_timeout(args.hdr, 30 + kEpi);
           *abort_flag = 1;
         }
         break;
@@ -263,6 +263,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_launch();
   tc_fence_before();
   __syncthreads();
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    // a role failed, possibly after the producer had finished: copies it
+    // issued that nobody consumed land before the CTA's memory goes away
+    for (int s = 0; s < kStages; ++s)
+      if (issued_mask & (1u << s)) (void)mbar_wait(&full[s], (last_phase >> s) & 1);
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

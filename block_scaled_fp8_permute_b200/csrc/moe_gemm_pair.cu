@@ -127,8 +127,7 @@ __global__ void __launch_bounds__(pairk::kThreads, 1)
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           if (!mbar_wait_cluster(&empty[s], ph ^ 1) || *abort_flag) {
-            set_status(args.hdr, MOE_ERR_TIMEOUT);
-            args.hdr[kHdrTimeoutSite] = 40 + kEpi;
+            record_timeout(args.hdr, 40 + kEpi);
             *abort_flag = 1;
             ok = false;
             break;
@@ -192,8 +191,7 @@ __global__ void __launch_bounds__(pairk::kThreads, 1)
         tc_commit_pair(acc_full, 0x3);
       }
       if (!ok) {
-        set_status(args.hdr, MOE_ERR_TIMEOUT);
-        args.hdr[kHdrTimeoutSite] = 50 + kEpi;
+        record_timeout(args.hdr, 50 + kEpi);
         *abort_flag = 1;
         if (issued_any) {  // wait for the MMAs in flight before TMEM is released
           tc_commit_pair(drain, 0x1);
@@ -217,8 +215,7 @@ __global__ void __launch_bounds__(pairk::kThreads, 1)
       const bool ready = __all_sync(0xffffffffu, mbar_wait(acc_full, ti & 1) && !*abort_flag);
       if (!ready) {
         if (lane == 0) {
-          set_status(args.hdr, MOE_ERR_TIMEOUT);
-          args.hdr[kHdrTimeoutSite] = 60 + kEpi;
+          record_timeout(args.hdr, 60 + kEpi);
           *abort_flag = 1;
         }
         break;

@@ -115,8 +115,7 @@ __global__ void __launch_bounds__(swapk::kThreads, 1)
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1) || *abort_flag) {
-            set_status(args.hdr, MOE_ERR_TIMEOUT);
-            args.hdr[kHdrTimeoutSite] = 70 + kEpi;
+            record_timeout(args.hdr, 70 + kEpi);
             *abort_flag = 1;
             ok = false;
             break;
@@ -189,8 +188,7 @@ __global__ void __launch_bounds__(swapk::kThreads, 1)
         tc_commit(acc_full);
       }
       if (!ok) {
-        set_status(args.hdr, MOE_ERR_TIMEOUT);
-        args.hdr[kHdrTimeoutSite] = 80 + kEpi;
+        record_timeout(args.hdr, 80 + kEpi);
         *abort_flag = 1;
         if (issued_any) {
           tc_commit(drain);
@@ -213,8 +211,7 @@ __global__ void __launch_bounds__(swapk::kThreads, 1)
       const bool ready = __all_sync(0xffffffffu, mbar_wait(acc_full, ti & 1) && !*abort_flag);
       if (!ready) {
         if (lane == 0) {
-          set_status(args.hdr, MOE_ERR_TIMEOUT);
-          args.hdr[kHdrTimeoutSite] = 90 + kEpi;
+          record_timeout(args.hdr, 90 + kEpi);
           *abort_flag = 1;
         }
         break;

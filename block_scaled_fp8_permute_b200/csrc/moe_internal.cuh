@@ -118,6 +118,12 @@ struct GemmArgs {
   uint16_t* d;
   const int* masked_m;
   int m_max;
+  // test hooks (moe_debug_set_fault), both off when 0: the wait limit of the
+  // MMA issuer's wait for a stage's data (the other waits of the kernel get
+  // twice this), and 1 + a pipeline iteration whose loads the producer of
+  // every CTA skips, so that the wait for that stage expires
+  unsigned long long wait_limit_ns;
+  int fault_skip_it;
 };
 
 // experts with at most this many routed rows use swapped operand roles
@@ -128,5 +134,14 @@ constexpr int kNarrowRows = 32;
 
 // record the first error of a call in the status word
 __device__ inline void set_status(int* hdr, int code) { atomicCAS(&hdr[kHdrStatus], 0, code); }
+
+// a bounded wait expired: MOE_ERR_TIMEOUT and the site of the first expiry
+// (10 + epilogue: producer, 20 + epilogue: MMA issuer, 30 + epilogue:
+// epilogue warps of the one-SM kernel; 40/50/60 + epilogue the same roles of
+// the SM-pair kernel, 70/80/90 + epilogue of the swapped-role kernel)
+__device__ inline void record_timeout(int* hdr, int site) {
+  set_status(hdr, MOE_ERR_TIMEOUT);
+  atomicCAS(&hdr[kHdrTimeoutSite], 0, site);
+}
 
 }  // namespace moe

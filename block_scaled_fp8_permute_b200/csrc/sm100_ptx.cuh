@@ -64,6 +64,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// The same wait with its own limit, which also gives up as soon as *abort is
+// non-zero (another role of the CTA has already failed).  Only for waits on
+// work that may never arrive: a wait for this CTA's own copies or MMAs in
+// flight must use mbar_wait, which returns only when they have landed.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity,
+                                                   unsigned long long limit_ns,
+                                                   const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort || globaltimer() - t0 > limit_ns) return false;
+  }
+}
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1) {

@@ -20,9 +20,11 @@
  *   a   = silu(g[0:I]) * g[I:2I]             (FP32; silu(z) = z / (1 + exp(-z)))
  *   a'  = E4M3 requantisation of a, one UE8M0 scale per 32 consecutive values,
  *         scale exponent = smallest e with 448 * 2^e >= amax (0 for amax 0)
- *   o   = W2[e] . a'                         (H outputs)
- *   p_s = BF16_RNE( topk_w[t][s] * o )       (the GEMM's BF16 output, section 4.3)
- *   y[t] = BF16_RNE( sum over s in slot order of p_s )                 (FP32 sum)
+ *   o_s = W2[e] . a'                         (H outputs)
+ *   y[t] = BF16_RNE( sum over s in slot order of topk_w[t][s] * o_s )
+ * (This implementation rounds each weighted slot output to BF16 and sums
+ * those in FP32 in slot order; against the definition, the error stays
+ * within normwise 5e-3 and 2e-2 * (|y| + rms(y)) per element.)
  * All products are block-scaled: every 1x32 block along K of x, W1, W2 and a'
  * carries one UE8M0 scale (value 2^(b-127)).
  *
@@ -108,8 +110,9 @@ void moe_set_gemm_variant(int variant);
  * swapped operand roles: the weights take the MMA's M side and the expert's
  * rows the N side (N = rows rounded up to 16), so a decode-sized expert no
  * longer pays for a 128-row tile ("DeepSeek DeepGEMM 2026年4月重磅更新" section
- * 8.1, Dynamic Swap A/B).  Read by moe_plan and moe_forward, which must see
- * the same value (set it before moe_plan); 0 disables.  Results are the same
+ * 8.1, Dynamic Swap A/B).  moe_plan takes the value current when it is
+ * called; changing it between moe_plan and moe_forward is safe (moe_forward
+ * runs every expert the plan listed).  0 disables.  Results are the same
  * either way.  Process-wide. */
 void moe_set_swap_max(int rows);
 
@@ -118,9 +121,9 @@ void moe_set_swap_max(int rows);
  * and so a deeper stream of the expert's weights (decode-sized batches are
  * bound by that stream).  -1 (default): on when the layer has at most 128
  * routed rows per expert on average; 0: off; 1: on.  Never with SM-pair
- * tiles.  Read by moe_plan and moe_forward, which must see the same value
- * (set it before moe_plan).  Results are the same either way.
- * Process-wide. */
+ * tiles.  moe_plan takes the value current when it is called; changing it
+ * between moe_plan and moe_forward is safe.  Results are the same either
+ * way.  Process-wide. */
 void moe_set_narrow_tiles(int mode);
 
 /* ---------------------------------------------------------------- weights */
@@ -194,11 +197,13 @@ moe_status moe_forward_host(const moe_shape* shape, const uint8_t* x_host,
                             void* workspace, size_t ws_bytes, moe_stream_t stream);
 
 /* ---------------------------------------------------- allocation-free call */
-/* The pages describe no counterpart of this entry point; it exists for
- * callers that cannot allocate device memory themselves: an inference
- * runtime whose memory manager owns every device byte, code that runs while
- * a CUDA graph is being captured, or a plug-in that is handed only its
- * inputs and outputs.  It performs moe_plan + moe_forward with the
+/* The pages describe no counterpart of this entry point.  It is for callers
+ * that cannot call cudaMalloc themselves: a serving runtime whose memory
+ * manager reserves the free device memory at start-up for its own pool (a
+ * further cudaMalloc would fail, or would take memory the pool counts on),
+ * or a plug-in / custom operator inside another framework that is handed
+ * only its input and output buffers and has no way to reach that
+ * framework's allocator for scratch space.  It performs moe_plan + moe_forward with the
  * workspace taken from a fixed 32 MiB array inside the library (a
  * file-scope __device__ array: every GPU that loads the library holds those
  * 32 MiB until the process exits).  The caller passes the inputs and y
@@ -228,6 +233,28 @@ moe_status moe_forward_noalloc(const moe_shape* shape, const uint8_t* x, const i
  * plan / forward that used `workspace` (MOE_OK, MOE_ERR_BAD_EXPERT_ID or
  * MOE_ERR_TIMEOUT), or MOE_ERR_CUDA if the stream itself failed. */
 moe_status moe_get_device_status(const void* workspace, moe_stream_t stream);
+
+/* Synchronises `stream` and returns where the first bounded device wait of
+ * the last forward on `workspace` expired: 0 none; 10 + j the TMA producer,
+ * 20 + j the MMA issuer, 30 + j the epilogue warps of the one-SM grouped
+ * GEMM, with j = 1 for linear1, 2 for linear2, 3 for the standalone GEMM;
+ * 40 + j, 50 + j, 60 + j the same roles in the SM-pair kernel; 70 + j,
+ * 80 + j, 90 + j in the swapped-role kernel.  -1 if the stream failed.
+ * Every wait on another role of the kernel is bounded (2 s for a stage's
+ * data, 4 s for the waits that can only end after such a stage); when one
+ * expires the kernel records MOE_ERR_TIMEOUT and this site, the other roles
+ * of the CTA stop waiting, copies and MMAs already in flight are waited for,
+ * tensor memory is freed and the kernel returns. */
+int moe_get_timeout_site(const void* workspace, moe_stream_t stream);
+
+/* Test hook for the failure path above (the pages' change list fixes a
+ * kernel hang; this checks that a wait which never ends is reported instead):
+ * in every following moe_forward, the producer of each CTA of the linear1
+ * kernel (one-SM tiles, normal m-tiles) skips the loads of its pipeline
+ * iteration `skip_iteration` (-1: off), and the waits of that kernel use
+ * `wait_limit_ns` for a stage's data and twice that otherwise (0: the
+ * defaults above).  Process-wide; both off by default. */
+void moe_debug_set_fault(int skip_iteration, unsigned long long wait_limit_ns);
 
 /* Copies the plan out of `workspace` for bit-exact checking (synchronises
  * `stream`).  All outputs are HOST buffers: counts [E], offs [E+1],
