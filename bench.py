@@ -6,8 +6,13 @@ linear2 x top-k weight -> combine) over one batch of the workload, inputs
 resident in HBM, L2 flushed (256 MB write) before every timed step.  Times
 are CUDA events on the launching stream.  Prints one JSON line (rank 0).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mid]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl ours|reference]
+
+Default: the headline is the largest config, the usage-example layer (T=8192,
+H=7168, I=9216, E=8, top-2); every other config (mid, skewed, decode at
+T=128/64/32/16) is measured the same way at N = 1 and reported under
+"configs" in the same line.  --workload NAME times NAME alone.
 
 Multi-GPU: replicas (each rank runs its own batch of the workload with its
 own activations; no collective on the data path); the step time is the max
@@ -57,7 +62,12 @@ def _args():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", default="mid")
+    p.add_argument("--workload", default=None,
+                   help="time only this workload (default: the usage config as the headline "
+                        "plus every other config as a sub-record)")
+    p.add_argument("--no-sub", action="store_true", help="headline only, no sub-records")
+    p.add_argument("--sub-cpu-seconds", type=float, default=4.0,
+                   help="target CPU time of each sub-record's oracle sample")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -265,17 +275,72 @@ def run_reference(args, wl, rank):
 
 
 # ------------------------------------------------------------------ ours
-def run_ours(args, wl, dist, rank, world, local_rank):
+# The headline workload (the largest config: the Mega MoE usage-example shape) and
+# the other configs, each measured the same way and reported as a sub-record of the
+# same JSON line.
+HEADLINE = "usage"
+SUB_WORKLOADS = ["mid", "skewed", "decode", "decode@T64", "decode@T32", "decode@T16"]
+GEN_WEIGHTS = {}   # (E, H, I, seed) -> host weights (skewed and decode share one layer)
+
+
+def _weights(wl):
+    key = (wl.E, wl.H, wl.I, wl.seed)
+    if key not in GEN_WEIGHTS:
+        import synth
+        GEN_WEIGHTS.clear()
+        GEN_WEIGHTS[key] = synth.make_weights(wl)
+    return GEN_WEIGHTS[key]
+
+
+def _roofline(wl, inputs, g1_ms, step_ms, pk, traffic):
+    """linear1's roofline (the slower of its FLOPs at the tensor peak and its
+    algorithmic bytes at the HBM peak) and the whole step's."""
+    import numpy as np
+    tensor_peak = 2.0 * pk["bf16"]  # FP8-rate MMA = 2 x the measured bf16 rate
+    hbm_peak = pk["hbm"]
+    # Algorithmic bytes: the weights of the experts that receive rows (FP4 codes +
+    # one UE8M0 byte per 32) are read once; activations, intermediate and output once.
+    idx = inputs["topk_idx"]
+    R_valid = int((idx >= 0).sum())
+    touched = len(np.unique(idx[idx >= 0]))
+    H, I = wl.H, wl.I
+    w1_bytes = touched * (2 * I * H // 2 + 2 * I * H // 32)
+    w2_bytes = touched * (H * I // 2 + H * I // 32)
+    g1_flops = 4.0 * R_valid * H * I
+    g1_bytes = w1_bytes + R_valid * (H + H // 32) + R_valid * (I + I // 32)
+    step_bytes = (w1_bytes + w2_bytes + wl.T * (H + H // 32) + wl.T * wl.k * 8 + wl.T * H * 2)
+    if g1_flops / (tensor_peak * 1e12) >= g1_bytes / (hbm_peak * 1e9):
+        roof = {"bound": "tensor", "achieved": g1_flops / (g1_ms * 1e-3) / 1e12,
+                "peak": tensor_peak, "unit": "TFLOP/s",
+                "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"}
+    else:
+        roof = {"bound": "hbm", "achieved": g1_bytes / (g1_ms * 1e-3) / 1e9, "peak": hbm_peak,
+                "unit": "GB/s", "peak_note": f"copy bandwidth {hbm_peak} GB/s ({pk['src']})"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof.update(kernel="linear1 (moe_gemm_kernel<1>, normal and narrow tiles)",
+                flops_per_launch=g1_flops, algorithmic_bytes_per_launch=g1_bytes,
+                traffic=traffic, traffic_unit="bytes per launch (ncu dram read+write)")
+    t_tensor = wl.flops / (tensor_peak * 1e12)
+    t_hbm = step_bytes / (hbm_peak * 1e9)
+    step = {"bound": "tensor" if t_tensor >= t_hbm else "hbm",
+            "roofline_ms": max(t_tensor, t_hbm) * 1e3, "frac": max(t_tensor, t_hbm) * 1e3 / step_ms,
+            "tflops": wl.flops / (step_ms * 1e-3) / 1e12,
+            "hbm_gbs": step_bytes / (step_ms * 1e-3) / 1e9,
+            "algorithmic_bytes": step_bytes, "experts_touched": touched}
+    return roof, step
+
+
+def measure(args, wl, inputs, dev, dist, weights=None, e2e=True):
+    """Time one workload: K replays of one captured plan + forward (L2 flushed
+    before each), then K eager steps with events at the kernel boundaries,
+    then (e2e) the host-buffer entry point.  Returns (record, layer)."""
     import numpy as np
     import torch
 
     import block_scaled_fp8_permute_b200 as moe
-    from tests.gpu_util import Layer
+    from block_scaled_fp8_permute_b200.layer import MoELayer
 
-    torch.cuda.set_device(local_rank)
-    dev = f"cuda:{local_rank}"
-    inputs = replica_inputs(wl, rank)  # shared weights, this replica's activations / routing
-    lay = Layer(inputs, device=dev)
+    lay = MoELayer(inputs, device=dev, weights=weights)
     shp, d = lay.shape, lay.dev
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -308,17 +373,16 @@ def run_ours(args, wl, dist, rank, world, local_rank):
         graph.replay()
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
     for row in kev:
         for e in row:
             e.record(stream)  # materialise the handles
+    if dist is not None:
+        dist.barrier()
     torch.cuda.synchronize()
     # clocks: sampled over the timed region (marked) and, as more evidence for a short
     # region, over the eager kernel-timing steps that follow it
-    clk = ClockSampler(local_rank)
+    clk = ClockSampler(torch.cuda.current_device())
     clk.__enter__()
     clk.wait_first()
     clk.mark("start")
@@ -333,6 +397,7 @@ def run_ours(args, wl, dist, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    del graph
 
     # Kernel durations: the same steps run eagerly with events at the kernel
     # boundaries (moe_set_timing_events), K more steps.
@@ -347,98 +412,140 @@ def run_ours(args, wl, dist, rank, world, local_rank):
     kern = {name: statistics.mean(kev[i][a].elapsed_time(kev[i][b]) for i in range(K))
             for name, a, b in (("plan", 0, 1), ("permute", 1, 2), ("linear1", 2, 3),
                                ("linear2", 3, 4), ("combine", 4, 5))}
-    ms = statistics.mean(step_ms)
     status = moe.moe_get_device_status(lay.ws)
     assert status == 0, f"device status {status}"
+    rec = {"ms": statistics.mean(step_ms), "ms_p50": statistics.median(step_ms),
+           "kernels_ms": kern, "clocks": clk.summary()}
 
-    # e2e: the host-buffer entry point, host<->device copies inside the timed region
-    ws_h = moe.alloc_workspace(shp, dev, host_variant=True)
-    pin = {k: torch.from_numpy(np.ascontiguousarray(inputs[k])).pin_memory()
-           for k in ("x", "x_sf", "topk_idx", "topk_w")}
-    y_host = torch.empty((wl.T, wl.H), dtype=torch.int16).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in pin.values())
-    d2h = y_host.numel() * y_host.element_size()
-    e2e_ms = []
-    for i in range(max(args.warmup, 3) + K):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        moe.moe_forward_host(shp, pin["x"], pin["x_sf"], pin["topk_idx"], pin["topk_w"], *lay.wt,
-                             y_host, ws_h)
-        e1.record(stream)
-        e1.synchronize()
-        if i >= max(args.warmup, 3):
-            e2e_ms.append(e0.elapsed_time(e1))
-    e2e = statistics.mean(e2e_ms)
+    if e2e:
+        # the host-buffer entry point, host<->device copies inside the timed region
+        ws_h = moe.alloc_workspace(shp, dev, host_variant=True)
+        pin = {k: torch.from_numpy(np.ascontiguousarray(inputs[k])).pin_memory()
+               for k in ("x", "x_sf", "topk_idx", "topk_w")}
+        y_host = torch.empty((wl.T, wl.H), dtype=torch.int16).pin_memory()
+        e2e_ms = []
+        for i in range(max(args.warmup, 3) + K):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            moe.moe_forward_host(shp, pin["x"], pin["x_sf"], pin["topk_idx"], pin["topk_w"],
+                                 *lay.wt, y_host, ws_h)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= max(args.warmup, 3):
+                e2e_ms.append(e0.elapsed_time(e1))
+        rec["e2e_ms"] = statistics.mean(e2e_ms)
+        rec["h2d"] = sum(t.numel() * t.element_size() for t in pin.values())
+        rec["d2h"] = y_host.numel() * y_host.element_size()
+        del ws_h
+    del flush
+    return rec, lay
 
-    ms = max_over_ranks(ms, dist, dev)
-    e2e = max_over_ranks(e2e, dist, dev)
-    g1 = max_over_ranks(kern["linear1"], dist, dev)
+
+def _launches_per_step(wl):
+    # count+scan, scatter, permute, linear1, linear2, combine; with narrow tiles (the
+    # library's default when the layer has <= 128 rows per expert) a second linear1
+    # and linear2 launch run the narrow m-tiles
+    return 6 + (2 if wl.R <= 128 * wl.E else 0)
+
+
+def _cpu_baseline(wl, inputs, seconds):
+    cv, n, sec, cores = _oracle_sample(wl, inputs, seconds)
+    return {"value": cv, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+            "tokens_per_s": n / sec,
+            "sample": f"{n} random tokens of {wl.T} (all top-{wl.k} slots), {sec:.1f} s"}
+
+
+def sub_record(args, wl, pk):
+    """One config measured at N = 1 as a sub-record of the headline line."""
+    import gc
+
+    import torch
+    x, x_sf, idx, tw = __import__("synth").make_activations(wl)
+    w1, w1_sf, w2, w2_sf = _weights(wl)
+    inputs = dict(x=x, x_sf=x_sf, topk_idx=idx, topk_w=tw, w1=w1, w1_sf=w1_sf, w2=w2, w2_sf=w2_sf)
+    key = (wl.E, wl.H, wl.I, wl.seed)
+    wt = SUB_DEVICE_WEIGHTS.get(key)
+    lay_inputs = dict(inputs, E=wl.E, I=wl.I) if wt is not None else inputs
+    rec, lay = measure(args, wl, lay_inputs, "cuda:0", None, weights=wt, e2e=True)
+    SUB_DEVICE_WEIGHTS.clear()
+    SUB_DEVICE_WEIGHTS[key] = lay.wt
+    roof, step = _roofline(wl, inputs, rec["kernels_ms"]["linear1"], rec["ms"], pk,
+                           _linear1_traffic(wl.name))
+    out = {"workload": _workload_desc(wl), "ms_per_step": rec["ms"], "ms_p50": rec["ms_p50"],
+           "tflops": wl.flops / (rec["ms"] * 1e-3) / 1e12,
+           "tokens_per_s": wl.T / (rec["ms"] * 1e-3), "roofline": roof, "step_roofline": step,
+           "kernels_ms": rec["kernels_ms"], "clocks": rec["clocks"],
+           "e2e": {"value": wl.flops / (rec["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
+                   "ms_per_step": rec["e2e_ms"], "h2d_bytes_per_step": rec["h2d"],
+                   "d2h_bytes_per_step": rec["d2h"]},
+           "gpu_launches_per_step": _launches_per_step(wl)}
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = _cpu_baseline(wl, inputs, args.sub_cpu_seconds)
+    del lay
+    gc.collect()
+    torch.cuda.empty_cache()
+    return out
+
+
+SUB_DEVICE_WEIGHTS = {}
+
+
+def run_ours(args, wl, dist, rank, world, local_rank):
+    import torch
+
+    torch.cuda.set_device(local_rank)
+    dev = f"cuda:{local_rank}"
+    inputs = replica_inputs(wl, rank)  # shared weights, this replica's activations / routing
+    rec, lay = measure(args, wl, inputs, dev, dist)
+    ms = max_over_ranks(rec["ms"], dist, dev)
+    e2e = max_over_ranks(rec["e2e_ms"], dist, dev)
+    g1 = max_over_ranks(rec["kernels_ms"]["linear1"], dist, dev)
+    del lay
+    subs = {}
+    if world == 1 and args.workload is None and not args.no_sub:
+        import gc
+        gc.collect()
+        torch.cuda.empty_cache()
+        pk = _peaks()
+        for name in SUB_WORKLOADS:
+            subs[name] = sub_record(args, __import__("synth").workload(name), pk)
     if rank != 0:
         return
     flops = wl.flops * world
     value = flops / (ms * 1e-3) / 1e12
     pk = _peaks()
-    tensor_peak = 2.0 * pk["bf16"]  # FP8-rate MMA = 2 x the measured bf16 rate
-    hbm_peak = pk["hbm"]
-    # Algorithmic bytes: the weights of the experts that receive rows (FP4 codes +
-    # one UE8M0 byte per 32) are read once; activations, intermediate and output once.
-    idx = inputs["topk_idx"]
-    R_valid = int((idx >= 0).sum())
-    touched = len(np.unique(idx[idx >= 0]))
-    H, I = wl.H, wl.I
-    w1_bytes = touched * (2 * I * H // 2 + 2 * I * H // 32)
-    w2_bytes = touched * (H * I // 2 + H * I // 32)
-    g1_flops = 4.0 * R_valid * H * I
-    g1_bytes = w1_bytes + R_valid * (H + H // 32) + R_valid * (I + I // 32)
-    step_bytes = (w1_bytes + w2_bytes + wl.T * (H + H // 32) + wl.T * wl.k * 8 + wl.T * H * 2)
-    # roofline time = the slower of the FLOPs at the tensor peak and the bytes at HBM bandwidth
-    g1_t_tensor = g1_flops / (tensor_peak * 1e12)
-    g1_t_hbm = g1_bytes / (hbm_peak * 1e9)
-    if g1_t_tensor >= g1_t_hbm:
-        roof = {"bound": "tensor", "achieved": g1_flops / (g1 * 1e-3) / 1e12, "peak": tensor_peak,
-                "unit": "TFLOP/s",
-                "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"}
-    else:
-        roof = {"bound": "hbm", "achieved": g1_bytes / (g1 * 1e-3) / 1e9, "peak": hbm_peak,
-                "unit": "GB/s", "peak_note": f"copy bandwidth {hbm_peak} GB/s ({pk['src']})"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    step_t_roof = max(wl.flops / (tensor_peak * 1e12), step_bytes / (hbm_peak * 1e9))
+    roof, step = _roofline(wl, inputs, g1, ms / 1.0, pk, _linear1_traffic(wl.name))
+    if world > 1:  # the step roofline of one replica (every rank runs the same shape)
+        step["note"] = "per replica"
     cpu = None
-    if not args.no_cpu_baseline:
-        cv, n, sec, cores = _oracle_sample(wl, inputs, args.cpu_seconds)
-        cpu = {"value": cv, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-               "sample": f"{n} random tokens of {wl.T} (all top-{wl.k} slots), {sec:.1f} s"}
+    if not args.no_cpu_baseline and world == 1:
+        cpu = _cpu_baseline(wl, inputs, args.cpu_seconds)
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOPS",
         "tokens_per_s": wl.T * world / (ms * 1e-3),
-        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8_e4m3 x fp4_e2m1, fp32 accumulate, bf16 out", "data": "synthetic",
         "config": {"workload": _workload_desc(wl), "tokens_per_gpu": wl.T,
                    "l2": "flushed (256 MB write) before every timed step",
                    "step": "moe_plan + moe_forward replayed as one CUDA graph",
                    "parallelism": f"replicas x{world}"},
-        "roofline": dict(roof, kernel="linear1 (moe_gemm_kernel<1>)",
-                         flops_per_launch=g1_flops, algorithmic_bytes_per_launch=g1_bytes,
-                         traffic=_linear1_traffic(wl.name),
-                         traffic_unit="bytes per launch (ncu dram read+write)"),
-        "kernels_ms": kern,
+        "roofline": roof,
+        "kernels_ms": rec["kernels_ms"],
         "kernels_ms_note": "eager steps with events at kernel boundaries (K extra steps)",
-        "step_roofline": {"bound": ("tensor" if wl.flops / (tensor_peak * 1e12)
-                                    >= step_bytes / (hbm_peak * 1e9) else "hbm"),
-                          "roofline_ms": step_t_roof * 1e3, "frac": step_t_roof * 1e3 / ms,
-                          "hbm_gbs": step_bytes / (ms * 1e-3) / 1e9,
-                          "algorithmic_bytes": step_bytes, "experts_touched": touched},
+        "step_roofline": step,
         "e2e": {"value": flops / (e2e * 1e-3) / 1e12, "unit": "TFLOPS",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
-        # count+scan, scatter, permute, linear1, linear2, combine; with narrow tiles (the
-        # library's default when the layer has <= 128 rows per expert) a second linear1
-        # and linear2 launch run the narrow m-tiles
-        "gpu_launches": (6 + (2 if wl.R <= 128 * wl.E else 0)) * K,
-        "clocks": clk.summary(),
+                "h2d_bytes_per_step": rec["h2d"], "d2h_bytes_per_step": rec["d2h"],
+                "ms_per_step": e2e},
+        "gpu_launches": _launches_per_step(wl) * args.steps,
+        "clocks": rec["clocks"],
         "cpu_baseline": cpu,
     }
+    if subs:
+        out["configs"] = subs
+        out["configs_note"] = ("the other configs, each measured at N = 1 like the headline "
+                               "(graph-replayed step, L2 flushed, CUDA events)")
     print(json.dumps(out), flush=True)
 
 
@@ -542,7 +649,7 @@ def main():
         if int(os.environ.get("RANK", "0")) == 0 and args.impl == "ours":
             run_gemm(args, args.workload)
         return
-    wl = synth.workload(args.workload)
+    wl = synth.workload(args.workload or HEADLINE)
     if args.impl == "reference":
         # the CPU oracle runs on rank 0 only; other ranks leave at once
         run_reference(args, wl, int(os.environ.get("RANK", "0")))

@@ -31,41 +31,8 @@ def assert_parity(y_gpu_bits, y_ref_bits, label=""):
     return p
 
 
-class Layer:
-    """Inputs of one workload on the device plus its transformed weights."""
-
-    def __init__(self, inputs: dict, device="cuda"):
-        import torch
-
-        import block_scaled_fp8_permute_b200 as moe
-        self.moe = moe
-        self.np = inputs
-        T, H = inputs["x"].shape
-        E, twoI, _ = inputs["w1"].shape
-        k = inputs["topk_idx"].shape[1]
-        self.shape = moe.shape(T, H, twoI // 2, E, k)
-        self.dev = {key: torch.from_numpy(np.ascontiguousarray(v)).to(device)
-                    for key, v in inputs.items()}
-        d = self.dev
-        self.wt = moe.transform_weights(self.shape, d["w1"], d["w1_sf"], d["w2"], d["w2_sf"])
-        self.ws = moe.alloc_workspace(self.shape, device)
-        self.y = torch.empty((max(T, 1), H), dtype=torch.bfloat16, device=device)
-
-    def run(self, topk_idx=None, topk_w=None, x=None, x_sf=None):
-        d = self.dev
-        idx = d["topk_idx"] if topk_idx is None else topk_idx
-        self.moe.moe_plan(self.shape, idx, self.ws)
-        self.moe.moe_forward(self.shape, d["x"] if x is None else x,
-                             d["x_sf"] if x_sf is None else x_sf, idx,
-                             d["topk_w"] if topk_w is None else topk_w, *self.wt, self.y,
-                             self.ws)
-        return self
-
-    def y_bits(self) -> np.ndarray:
-        import torch
-        torch.cuda.synchronize()
-        T = self.shape.T
-        return self.y[:T].view(torch.int16).cpu().numpy().view(np.uint16)
-
-    def status(self) -> int:
-        return self.moe.moe_get_device_status(self.ws)
+def Layer(inputs: dict, device="cuda"):
+    """The package's device-resident layer (imported here, not at module load, so
+    that collecting the GPU tests on a machine without the built library works)."""
+    from block_scaled_fp8_permute_b200.layer import MoELayer
+    return MoELayer(inputs, device=device)

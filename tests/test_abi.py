@@ -11,8 +11,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def moe():
-    from block_scaled_fp8_permute_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()          # builds before the package loads the library
     import block_scaled_fp8_permute_b200 as m
     return m
 
