@@ -1,6 +1,9 @@
 // moe_noalloc.cu -- the allocation-free entry point: plan + forward of one
 // MoE layer with the workspace taken from a fixed device array that the
-// library itself owns, for callers that cannot allocate device memory.
+// library itself owns.  It serves callers that cannot call cudaMalloc: a
+// serving runtime whose memory manager has reserved the free device memory
+// for its own pool, or a plug-in that is handed only its inputs and outputs
+// and cannot reach its host framework's allocator.
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -44,6 +47,7 @@ moe_status moe_forward_noalloc(const moe_shape* shape, const uint8_t* x, const i
                                const int32_t* topk_idx, const float* topk_w, const void* w1_t,
                                const void* w1_sf_t, const void* w2_t, const void* w2_sf_t,
                                uint16_t* y, moe_stream_t stream) {
+  if (!shape) return MOE_ERR_INVALID_ARG;  // as moe_forward
   const size_t need = moe_workspace_bytes(shape);
   if (need == 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (need > moe::kStaticScratchBytes) return MOE_ERR_WORKSPACE;

@@ -1,9 +1,11 @@
-"""The allocation-free entry point, moe_forward_noalloc, for callers that
-cannot allocate device memory (a runtime whose allocator owns all device
-memory, code running under CUDA-graph capture, a plug-in handed only its
-inputs and outputs).  It must give what moe_forward gives, on two calls in a
-row (the second reuses the library's fixed workspace with its previous
-contents), and must reject shapes whose workspace exceeds its 32 MiB array.
+"""The allocation-free entry point, moe_forward_noalloc.  It is for callers
+that cannot call cudaMalloc: a serving runtime whose memory manager has
+reserved the free device memory for its own pool, or a plug-in handed only
+its input and output buffers with no access to its host framework's
+allocator.  It must give what moe_forward gives (and stay within the
+oracle's tolerance) on two calls in a row, the second reusing the library's
+fixed workspace with the previous call's contents, and must reject shapes
+whose workspace exceeds its 32 MiB array.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test."""
@@ -12,6 +14,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 import synth
 from tests.gpu_util import Layer, assert_parity
 
@@ -43,6 +46,8 @@ def test_noalloc_matches_forward_on_two_calls():
     y_ref = lay.y_bits()
     y1 = _noalloc(lay, moe)
     assert_parity(y1, y_ref, "noalloc call 1")
+    y_orc, _, _ = oracle.moe_forward(**d)
+    assert_parity(y1, y_orc, "noalloc call 1 vs oracle")
     # a second call with a different routing, then the original again: the
     # fixed workspace keeps the previous call's contents in between
     import torch
@@ -59,3 +64,4 @@ def test_noalloc_rejects_oversized_shapes():
     assert moe.moe_workspace_bytes(shp) > (32 << 20)
     st = moe.lib().moe_forward_noalloc(ctypes.byref(shp), *([None] * 9), None)
     assert st == 3                                      # MOE_ERR_WORKSPACE, nothing launched
+    assert moe.lib().moe_forward_noalloc(None, *([None] * 9), None) == 1   # as moe_forward
