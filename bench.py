@@ -69,6 +69,11 @@ def _args():
     p.add_argument("--sub-cpu-seconds", type=float, default=4.0,
                    help="target CPU time of each sub-record's oracle sample")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--gemm-variant", type=int, default=None,
+                   help="moe_set_gemm_variant before timing (0 one-SM tiles, 1 SM pairs)")
+    p.add_argument("--swap-max", type=int, default=None, help="moe_set_swap_max before timing")
+    p.add_argument("--narrow", type=int, default=None,
+                   help="moe_set_narrow_tiles before timing (-1 auto, 0 off, 1 on)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the bounded oracle sample")
@@ -655,6 +660,14 @@ def main():
         run_reference(args, wl, int(os.environ.get("RANK", "0")))
         return
     dist, rank, world, local_rank = _dist()
+    if args.gemm_variant is not None or args.swap_max is not None or args.narrow is not None:
+        import block_scaled_fp8_permute_b200 as moe
+        if args.gemm_variant is not None:
+            moe.moe_set_gemm_variant(args.gemm_variant)
+        if args.swap_max is not None:
+            moe.moe_set_swap_max(args.swap_max)
+        if args.narrow is not None:
+            moe.moe_set_narrow_tiles(args.narrow)
     try:
         run_ours(args, wl, dist, rank, world, local_rank)
     finally:

@@ -8,9 +8,9 @@
 #include "moe_internal.cuh"
 
 namespace moe {
-cudaError_t launch_gemm(int epi, bool narrow, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                        const CUtensorMap& tmOut, const GemmArgs& args, int grid, bool pdl,
-                        cudaStream_t stream);
+cudaError_t launch_gemm(int epi, bool narrow, const CUtensorMap& tmA, const CUtensorMap& tmAn,
+                        const CUtensorMap& tmB, const CUtensorMap& tmOut, const GemmArgs& args,
+                        int grid, bool pdl, cudaStream_t stream);
 cudaError_t launch_gemm_pair(int epi, const CUtensorMap& tmA, const CUtensorMap& tmB,
                              const CUtensorMap& tmSFA, const CUtensorMap& tmSFB,
                              const CUtensorMap& tmOut, const GemmArgs& args, int num_pairs_grid,
@@ -278,7 +278,7 @@ moe_status gemm_run(int G, int M_max, int N, int K, const uint8_t* a, const int3
   const long long tiles = (long long)L.MT * NT;
   const int grid = (int)(tiles < sms ? tiles : sms);
   return cuda_status(
-      launch_gemm(3, false, tmA, tmB, tmD, g, grid < 1 ? 1 : grid, g_pdl.load() != 0, s));
+      launch_gemm(3, false, tmA, tmA, tmB, tmD, g, grid < 1 ? 1 : grid, g_pdl.load() != 0, s));
 }
 
 // staging area of moe_forward_host, after the regular workspace
@@ -494,6 +494,15 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   g1.a2_sf = ws.a2_sf();
   g1.I = sh.I;
   g1.H = sh.H;
+  g1.narrow_mtiles = ws.narrow_mt();
+  // experts with at most kNarrowRows rows: narrow tiles (a deeper weight stream).
+  // Launched whenever the plan may have listed such experts, whatever the knobs
+  // say now (an empty list costs one short launch).  With one-SM normal tiles
+  // the launches are mixed: the normal-tile kernel also runs the narrow m-tiles
+  // when the plan has normal m-tiles too, so their weight streams overlap the
+  // compute-bound tiles; otherwise the narrow-tile kernel runs them.
+  const bool narrow = narrow_possible(sh);
+  g1.mixed = (narrow && !pair1) ? 1 : 0;
   GemmArgs g1f = g1;  // the normal one-SM linear1 launch carries the test hook
   g1f.fault_skip_it = g_fault_skip_it.load();
   g1f.wait_limit_ns = g_fault_wait_ns.load();
@@ -504,20 +513,16 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   } else {
     long long tiles1 = (long long)ws.L.MT_max * NT1;
     int grid1 = (int)(tiles1 < sms ? tiles1 : sms);
-    e = launch_gemm(1, false, tmX, tmW1, tmYp, g1f, grid1 < 1 ? 1 : grid1, pdl, s);
+    e = launch_gemm(1, false, tmX, tmXn, tmW1, tmYp, g1f, grid1 < 1 ? 1 : grid1, pdl, s);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  // experts with at most kNarrowRows rows: narrow tiles (a deeper weight stream).
-  // Launched whenever the plan may have listed such experts, whatever the knobs
-  // say now (an empty list costs one short launch).
-  const bool narrow = narrow_possible(sh);
   const int narrow_grid1 = (int)((long long)sh.E * NT1 < sms ? (long long)sh.E * NT1 : sms);
   if (narrow) {
     GemmArgs g1n = g1;
     g1n.norm_mtiles = ws.narrow_mt();
     g1n.tiles_word = kHdrNarrowMTiles;
     // 256-row weight boxes, whatever box the SM-pair tiles use
-    e = launch_gemm(1, true, tmXn, tmW1s, tmYp, g1n, narrow_grid1, pdl, s);
+    e = launch_gemm(1, true, tmXn, tmXn, tmW1s, tmYp, g1n, narrow_grid1, pdl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
   // swapped-role tiles exist only when the plan was made with a threshold > 0
@@ -537,6 +542,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   g2.NT = NT2;
   g2.yp = ws.yp();
   g2.topk_w = topk_w;
+  g2.mixed = (narrow && !pair2) ? 1 : 0;
   if (pair2) {
     long long work = (long long)ws.L.MP_max * NT2;
     int pairs = (int)(work < max_pairs_grid ? work : max_pairs_grid);
@@ -544,7 +550,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
   } else {
     long long tiles2 = (long long)ws.L.MT_max * NT2;
     int grid2 = (int)(tiles2 < sms ? tiles2 : sms);
-    e = launch_gemm(2, false, tmA2, tmW2, tmYp, g2, grid2 < 1 ? 1 : grid2, pdl, s);
+    e = launch_gemm(2, false, tmA2, tmA2n, tmW2, tmYp, g2, grid2 < 1 ? 1 : grid2, pdl, s);
   }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   if (narrow) {
@@ -552,7 +558,7 @@ moe_status moe_forward(const moe_shape* shape, const uint8_t* x, const int32_t* 
     g2n.norm_mtiles = ws.narrow_mt();
     g2n.tiles_word = kHdrNarrowMTiles;
     const int narrow_grid2 = (int)((long long)sh.E * NT2 < sms ? (long long)sh.E * NT2 : sms);
-    e = launch_gemm(2, true, tmA2n, tmW2s, tmYp, g2n, narrow_grid2, pdl, s);
+    e = launch_gemm(2, true, tmA2n, tmA2n, tmW2s, tmYp, g2n, narrow_grid2, pdl, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
   if (use_swap) {

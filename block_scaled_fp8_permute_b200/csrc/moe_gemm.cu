@@ -33,6 +33,11 @@ namespace moe {
 
 constexpr int kSmemB = kBlockN * kBlockK;  // 32768 bytes (one byte per E2M1 element in smem)
 constexpr int kTxB = kBlockN * kBlockK / 2;  // bytes the TMA moves for B (packed)
+// Scale factors of one stage: the 512-byte chunk of A's 128 rows and the two
+// chunks of B's 256 rows, copied into TMEM by tcgen05.cp .32x128b.warpx4
+// (the layout the block-scaled MMA reads: every 32-lane subpartition holds
+// all rows).  (Copies without replication from four replicas per chunk are
+// cheaper in the tensor pipe, but the extra loads per stage cost more.)
 constexpr int kSmemSFA = kSfChunk;
 constexpr int kSmemSFB = 2 * kSfChunk;
 constexpr int kNumEpiWarps = 8;
@@ -40,6 +45,7 @@ constexpr int kGemmThreads = 64 + 32 * kNumEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;    // FP32 accumulator, 256 columns
 constexpr uint32_t kSfCol = 256;   // scale buffers: buf b -> SFA at +16b (4 cols), SFB at +16b+4 (8)
+
 constexpr int kOutStage = kEpiOutStage;
 
 // Stage geometry.  Normal tiles stage 128 A rows (16 KB) per 128-K step in a
@@ -49,15 +55,21 @@ constexpr int kOutStage = kEpiOutStage;
 // still spans 128 rows: rows past kNarrowRows read whatever the shared memory
 // after the stage's A rows holds, and those accumulator rows (padding) are
 // never stored.
-template <bool kNarrow>
+template <int kEpi, bool kNarrow>
 struct TileCfg {
   static constexpr int kARows = kNarrow ? kNarrowRows : kBlockM;
   static constexpr int kStages = kNarrow ? 5 : 4;
   static constexpr int kSmemA = kARows * kBlockK;
-  static constexpr size_t kSmemBytes =
-      1024 + (size_t)kStages * (kSmemA + kSmemB + kSmemSFA + kSmemSFB) +
-      (size_t)kNumEpiWarps * kOutStage + 256;
+  static constexpr int kStageBytes = kSmemA + kSmemB + kSmemSFA + kSmemSFB;
+  static constexpr int kOutBytes = kEpi == 1 ? 0 : kNumEpiWarps * kOutStage;
+  // the dynamic shared memory base is 1024-byte aligned (checked at kernel start)
+  static constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + kOutBytes + 256;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  // A and B stage buffers keep the 1024-byte alignment of the 128-byte
+  // swizzle; the epilogue staging after all stage arrays the 512 bytes of the
+  // 64-byte swizzle
+  static_assert(kSmemA % 1024 == 0 && kSmemB % 1024 == 0, "swizzled stage alignment");
+  static_assert(((size_t)kStages * kStageBytes) % 512 == 0, "staging alignment");
 };
 
 __global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int cols,
@@ -78,25 +90,53 @@ __global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int 
   }
 }
 
+// Tile v of a launch with `total` tiles of which `n_mix` are mixed-in narrow
+// tiles: narrow tiles sit at the positions where floor(v * n_mix / total)
+// steps up, so they are spread evenly over the launch and every CTA (which
+// takes every gridDim-th tile) gets its share.  Returns true for a narrow
+// tile; mt / nt: its m-tile and n-tile.
+__device__ __forceinline__ bool decode_tile(int v, int total, int n_mix, int NT,
+                                            const GemmArgs& args, int& mt, int& nt) {
+  if (n_mix == 0) {
+    mt = args.norm_mtiles[v / NT];
+    nt = v - (v / NT) * NT;
+    return false;
+  }
+  const long long before = (long long)v * n_mix / total;          // narrow tiles before v
+  const long long upto = ((long long)v + 1) * n_mix / total;      // ... up to and with v
+  const bool nar = upto > before;
+  const int idx = nar ? (int)before : v - (int)before;
+  const int* list = nar ? args.narrow_mtiles : args.norm_mtiles;
+  mt = list[idx / NT];
+  nt = idx - (idx / NT) * NT;
+  return nar;
+}
+
 // -------------------------------------------------------------------- kernel
 template <int kEpi,    // 1: SwiGLU + requant (linear1), 2: x topk_w, BF16 rows (linear2),
                        // 3: BF16 rows of the standalone GEMM
           bool kNarrow>  // stage only kNarrowRows A rows (TileCfg)
 __global__ void __launch_bounds__(kGemmThreads, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmAn,  // kNarrowRows-row A boxes
                     const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmOut, const GemmArgs args) {
   using namespace ptx;
-  constexpr int kStages = TileCfg<kNarrow>::kStages;
-  constexpr int kSmemA = TileCfg<kNarrow>::kSmemA;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<size_t>(smem_raw), 1024));
+  using Cfg = TileCfg<kEpi, kNarrow>;
+  constexpr int kStages = Cfg::kStages;
+  constexpr int kSmemA = Cfg::kSmemA;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // the layout below needs it; no work done yet
+    if (threadIdx.x == 0) set_status(args.hdr, MOE_ERR_CUDA);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sA = smem;
   uint8_t* sB = sA + kStages * kSmemA;
   uint8_t* sSFA = sB + kStages * kSmemB;
   uint8_t* sSFB = sSFA + kStages * kSmemSFA;
   uint8_t* sOut = sSFB + kStages * kSmemSFB;  // epilogue staging, 1024-aligned
-  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kNumEpiWarps * kOutStage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sOut + Cfg::kOutBytes);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 1;
@@ -136,7 +176,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // end after such a stage (free slots, the accumulator) get 2L, so that the
   // wait nearest the cause expires first
   const unsigned long long lim = args.wait_limit_ns ? args.wait_limit_ns : kWaitLimitNs;
-  const int num_tiles = args.hdr[args.tiles_word] * NT;
+  // tiles of this launch: its own list, plus (mixed normal-tile launch) the
+  // narrow m-tiles spread evenly among them; a mixed narrow-tile launch has
+  // nothing to do when the normal-tile launch took its tiles
+  const int n_norm_mt = args.hdr[kHdrNormMTiles];
+  int n_own = args.hdr[args.tiles_word] * NT, n_mix = 0;
+  if (args.mixed) {
+    if (kNarrow && n_norm_mt > 0) n_own = 0;
+    if (!kNarrow && n_norm_mt > 0) n_mix = args.hdr[kHdrNarrowMTiles] * NT;
+  }
+  const int num_tiles = n_own + n_mix;
 
   // stages the producer has issued loads into, and the phase of the last one
   // (producer lane only): after a failure they are waited for before exit
@@ -147,11 +196,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int mt = args.norm_mtiles[tile / NT], nt = tile - (tile / NT) * NT;
+        int mt, nt;
+        const bool nar = decode_tile(tile, num_tiles, n_mix, NT, args, mt, nt);
         const int e = args.tile_expert[mt];
         const int n0 = nt * kBlockN;
-        const uint32_t sfb_bytes = (n_rows - n0 > 128) ? 2 * kSfChunk : kSfChunk;
-        const uint32_t tx = kSmemA + kTxB + kSfChunk + sfb_bytes;
+        const bool two_chunks = n_rows - n0 > 128;  // 256 weight rows (else the 128-row tail)
+        const uint32_t a_bytes = nar ? kNarrowRows * kBlockK : kSmemA;
+        const uint32_t tx = a_bytes + kTxB + kSfChunk + (two_chunks ? 2 : 1) * kSfChunk;
         const uint8_t* sfa_src = args.sfa + (size_t)mt * KB * kSfChunk;
         const uint8_t* sfb_src = args.sfb + ((size_t)e * KB * (n_rows / 128) + n0 / 128) * kSfChunk;
         for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -165,11 +216,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           if ((int)it + 1 == args.fault_skip_it) continue;  // test hook: this stage never fills
           mbar_arrive_expect_tx(&full[s], tx);
-          tma_load_2d(sA + s * kSmemA, &tmA, &full[s], kb * kBlockK, mt * kBlockM);
+          tma_load_2d(sA + s * kSmemA, nar ? &tmAn : &tmA, &full[s], kb * kBlockK, mt * kBlockM);
           tma_load_3d(sB + s * kSmemB, &tmB, &full[s], 0, n0, e * KB + kb);
           bulk_load(sSFA + s * kSmemSFA, sfa_src + (size_t)kb * kSfChunk, kSfChunk, &full[s]);
           bulk_load(sSFB + s * kSmemSFB, sfb_src + (size_t)kb * (n_rows / 128) * kSfChunk,
-                    sfb_bytes, &full[s]);
+                    (two_chunks ? 2 : 1) * kSfChunk, &full[s]);
           issued_mask |= 1u << s;
           last_phase = (last_phase & ~(1u << s)) | (ph << s);
         }
@@ -181,8 +232,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t it = 0;
       int ti = 0;
       bool issued_any = false, ok = true;
+      // descriptors of stage 0; stage s adds its byte offset >> 4 to the start field
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA)), b_desc0 = sdesc_sw128(smem_u32(sB));
+      const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++ti) {
-        const int nt = tile % NT;
+        int mt, nt;
+        (void)decode_tile(tile, num_tiles, n_mix, NT, args, mt, nt);
         const int n_tile = min(kBlockN, n_rows - nt * kBlockN);
         const uint32_t idesc0 = idesc_mxf8f6f4(/*A E4M3*/ 0, /*B E2M1*/ 5, kBlockM, n_tile);
         if (!mbar_wait_or_abort(acc_empty, (ti & 1) ^ 1, 2 * lim, abort_flag)) {
@@ -200,12 +255,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t sfa_t = tmem + kSfCol + 16u * (it & 1u);
           const uint32_t sfb_t = sfa_t + 4u;
-          tc_cp_32x128b_warpx4(sfa_t, sdesc_sf(smem_u32(sSFA + s * kSmemSFA)));
-          tc_cp_32x128b_warpx4(sfb_t, sdesc_sf(smem_u32(sSFB + s * kSmemSFB)));
+          tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + (uint64_t)((s * kSmemSFA) >> 4));
+          tc_cp_32x128b_warpx4(sfb_t, sfb_desc0 + (uint64_t)((s * kSmemSFB) >> 4));
           if (n_tile > 128)
-            tc_cp_32x128b_warpx4(sfb_t + 4u, sdesc_sf(smem_u32(sSFB + s * kSmemSFB + kSfChunk)));
-          const uint64_t adesc = sdesc_sw128(smem_u32(sA + s * kSmemA));
-          const uint64_t bdesc = sdesc_sw128(smem_u32(sB + s * kSmemB));
+            tc_cp_32x128b_warpx4(sfb_t + 4u, sfb_desc0 + (uint64_t)((s * kSmemSFB + kSfChunk) >> 4));
+          const uint64_t adesc = a_desc0 + (uint64_t)((s * kSmemA) >> 4);
+          const uint64_t bdesc = b_desc0 + (uint64_t)((s * kSmemB) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t id = idesc_with_sf_id(idesc0, kk, kk);
@@ -237,7 +292,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + kAccCol;
     int ti = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++ti) {
-      const int mt = args.norm_mtiles[tile / NT], nt = tile - (tile / NT) * NT;
+      int mt, nt;
+      (void)decode_tile(tile, num_tiles, n_mix, NT, args, mt, nt);
       // warp-uniform decision: every lane leaves or every lane continues
       const bool ready =
           __all_sync(0xffffffffu, mbar_wait_or_abort(acc_full, ti & 1, 2 * lim, abort_flag));
@@ -277,21 +333,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ------------------------------------------------------------ host launchers
-cudaError_t launch_gemm(int epi, bool narrow, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                        const CUtensorMap& tmOut, const GemmArgs& args, int grid, bool pdl,
-                        cudaStream_t stream) {
-  typedef void (*Fn)(CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs);
+cudaError_t launch_gemm(int epi, bool narrow, const CUtensorMap& tmA, const CUtensorMap& tmAn,
+                        const CUtensorMap& tmB, const CUtensorMap& tmOut, const GemmArgs& args,
+                        int grid, bool pdl, cudaStream_t stream) {
+  typedef void (*Fn)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs);
   static bool attr_set[2][4] = {};
   Fn fn;
   size_t smem;
   if (narrow) {
     if (epi != 1 && epi != 2) return cudaErrorInvalidValue;
     fn = epi == 1 ? moe_gemm_kernel<1, true> : moe_gemm_kernel<2, true>;
-    smem = TileCfg<true>::kSmemBytes;
+    smem = epi == 1 ? TileCfg<1, true>::kSmemBytes : TileCfg<2, true>::kSmemBytes;
   } else {
     fn = epi == 1 ? moe_gemm_kernel<1, false>
                   : (epi == 2 ? moe_gemm_kernel<2, false> : moe_gemm_kernel<3, false>);
-    smem = TileCfg<false>::kSmemBytes;
+    smem = epi == 1 ? TileCfg<1, false>::kSmemBytes
+                    : (epi == 2 ? TileCfg<2, false>::kSmemBytes : TileCfg<3, false>::kSmemBytes);
   }
   if (!attr_set[narrow][epi]) {
     cudaError_t err =
@@ -309,7 +366,7 @@ cudaError_t launch_gemm(int epi, bool narrow, const CUtensorMap& tmA, const CUte
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, fn, tmA, tmB, tmOut, args);
+  return cudaLaunchKernelEx(&cfg, fn, tmA, tmAn, tmB, tmOut, args);
 }
 
 cudaError_t launch_requant_debug(const float* a, int rows, int cols, uint8_t* codes,

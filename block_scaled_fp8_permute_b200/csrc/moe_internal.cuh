@@ -118,6 +118,13 @@ struct GemmArgs {
   uint16_t* d;
   const int* masked_m;
   int m_max;
+  // mixed launches (one-SM tiles, layers with both large and narrow-tiled
+  // experts): the normal-tile kernel also runs the narrow m-tiles, spread
+  // evenly among its own, when the plan listed normal m-tiles, and the
+  // narrow-tile kernel then has nothing to do; without normal m-tiles the
+  // narrow-tile kernel runs them (its deeper ring suits a pure weight stream)
+  int mixed;
+  const int* narrow_mtiles;
   // test hooks (moe_debug_set_fault), both off when 0: the wait limit of the
   // MMA issuer's wait for a stage's data (the other waits of the kernel get
   // twice this), and 1 + a pipeline iteration whose loads the producer of
