@@ -71,6 +71,13 @@ def _load():
     lib.orc_gemm.restype = None
     lib.orc_gemm.argtypes = ([ctypes.c_int] * 4 + [c_u8p, c_i32p, c_i32p, c_u8p, c_u8p,
                                                    ctypes.POINTER(ctypes.c_uint16), ctypes.c_int])
+    lib.orc_mqa_logits.restype = None
+    lib.orc_mqa_logits.argtypes = ([ctypes.c_int] * 4 + [c_u8p, c_i32p, c_u8p, c_u8p,
+                                                          ctypes.POINTER(ctypes.c_float), c_i32p,
+                                                          c_i32p, ctypes.c_int,
+                                                          ctypes.POINTER(ctypes.c_float),
+                                                          ctypes.POINTER(ctypes.c_double),
+                                                          ctypes.c_int])
     lib.orc_max_threads.restype = ctypes.c_int
     lib.orc_max_threads.argtypes = []
     _lib = lib
@@ -207,6 +214,31 @@ def gemm(a, a_sf, b, b_sf, masked_m=None, out=None, nthreads=0):
                      _ptr(b3, ctypes.c_uint8), _ptr(bs3, ctypes.c_uint8),
                      _ptr(d, ctypes.c_uint16), int(nthreads))
     return d[0] if dense else d
+
+
+def mqa_logits(q, q_sf, kv, kv_sf, weights, ks, ke, clean=True, want_mag=False, nthreads=0):
+    """FP4-indexer logits, float32 [S, N] (entries outside [ks, ke) are -inf
+    when clean, else NaN as 'not written').  q u8 [S, Hh, D]; q_sf i32
+    [S, Hh, D/128]; kv u8 [N, D/2]; kv_sf u8 [N, D/32]; weights f32 [S, Hh];
+    ks, ke i32 [S].  Returns (logits, mag or None)."""
+    q = np.ascontiguousarray(q, np.uint8)
+    S, Hh, D = q.shape
+    N = kv.shape[0]
+    arrs = [np.ascontiguousarray(a) for a in (q_sf, kv, kv_sf)]
+    q_sf, kv, kv_sf = arrs
+    w = np.ascontiguousarray(weights, np.float32)
+    ks = np.ascontiguousarray(ks, np.int32)
+    ke = np.ascontiguousarray(ke, np.int32)
+    assert q_sf.dtype == np.int32 and kv.dtype == np.uint8 and kv_sf.dtype == np.uint8
+    out = np.full((S, N), np.nan, np.float32)
+    mag = np.zeros((S, N), np.float64) if want_mag else None
+    _load().orc_mqa_logits(S, Hh, D, N, _ptr(q, ctypes.c_uint8), _ptr(q_sf, ctypes.c_int32),
+                           _ptr(kv, ctypes.c_uint8), _ptr(kv_sf, ctypes.c_uint8),
+                           _ptr(w, ctypes.c_float), _ptr(ks, ctypes.c_int32),
+                           _ptr(ke, ctypes.c_int32), 1 if clean else 0,
+                           _ptr(out, ctypes.c_float),
+                           _ptr(mag, ctypes.c_double) if mag is not None else None, int(nthreads))
+    return out, mag
 
 
 def max_threads() -> int:

@@ -345,3 +345,65 @@ int orc_max_threads(void) {
   return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------ */
+/* FP4 indexer: MQA logits with FP8 queries and FP4 keys ([EXPLAINER] 5.1   */
+/* and 5.2, the fp8_fp4_mqa_logits call; [NEWS] "FP4 Indexer").             */
+/* ------------------------------------------------------------------------ */
+/* Readings (each with its reason in the design notes):
+ *   - q is FP8 E4M3 and kv is FP4 E2M1, both with one UE8M0 scale per 1x32
+ *     block along the head dimension (the library's fp8_fp4_* naming: FP8
+ *     first operand, FP4 second);
+ *   - logits[i][j] = sum_h weights[i][h] * max(0, sum_d q[i][h][d] * k[j][d])
+ *     (the page's formula has a two-index logit and per-head weights; the
+ *     softmax inside its ReLU is dropped);
+ *   - only keys ks[i] <= j < ke[i] are scored; with clean != 0 every other
+ *     entry of row i is -inf, otherwise it is not written;
+ *   - the output is FP32 (the cleaned entries are -inf, which no FP4 code
+ *     holds).
+ * Layouts: q u8 [S, Hh, D] E4M3; q_sf i32 [S, Hh, D/128] (byte j of word i =
+ * scale of block 4i+j, as x_sf); kv u8 [N, D/2] E2M1 (low nibble = even d);
+ * kv_sf u8 [N, D/32]; weights f32 [S, Hh]; ks, ke i32 [S]; logits f32 [S, N].
+ * When mag is not NULL, mag[i][j] = sum_h |weights[i][h] * dot_h| (a bound
+ * on the size of every term, used to scale the comparison tolerance). */
+void orc_mqa_logits(int S, int Hh, int D, int N, const uint8_t* q, const int32_t* q_sf,
+                    const uint8_t* kv, const uint8_t* kv_sf, const float* weights,
+                    const int32_t* ks, const int32_t* ke, int clean, float* logits, double* mag,
+                    int nthreads) {
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int i = 0; i < S; ++i) {
+    double* qd = (double*)malloc(sizeof(double) * (size_t)Hh * D);
+    double* kd = (double*)malloc(sizeof(double) * (size_t)D);
+    for (int h = 0; h < Hh; ++h)
+      for (int d = 0; d < D; ++d)
+        qd[(size_t)h * D + d] = x_value(q, q_sf, D, i * Hh + h, d);
+    int lo = ks[i] < 0 ? 0 : ks[i];
+    int hi = ke[i] > N ? N : ke[i];
+    for (int j = 0; j < N; ++j) {
+      float* out = logits + (size_t)i * N + j;
+      if (j < lo || j >= hi) {
+        if (clean) *out = -INFINITY;
+        if (mag) mag[(size_t)i * N + j] = 0.0;
+        continue;
+      }
+      for (int d = 0; d < D; ++d) kd[d] = w_value(kv, kv_sf, N, D, 0, j, d);
+      double acc = 0.0, m = 0.0;
+      for (int h = 0; h < Hh; ++h) {
+        double s = 0.0;
+        for (int d = 0; d < D; ++d) s += qd[(size_t)h * D + d] * kd[d];
+        double w = (double)weights[(size_t)i * Hh + h];
+        if (s > 0.0) acc += w * s;
+        m += fabs(w * s);
+      }
+      *out = (float)acc;
+      if (mag) mag[(size_t)i * N + j] = m;
+    }
+    free(qd);
+    free(kd);
+  }
+}

@@ -126,3 +126,18 @@ def moe_masked(x, x_sf, topk_idx, topk_w, w1, w1_sf, w2, w2_sf):
             sel = (topk_idx[:, s] == e).astype(np.float64) * topk_w[:, s].astype(np.float64)
             acc += sel[:, None] * O
     return acc
+
+
+def mqa_logits(q, q_sf, kv, kv_sf, weights, ks, ke):
+    """FP4-indexer logits written independently: decode q and k to float64,
+    per-head dot products as one matmul, ReLU, weighted head sum; entries
+    outside [ks, ke) are -inf.  Returns float64 [S, N]."""
+    S, Hh, D = q.shape
+    N = kv.shape[0]
+    Q = dequant_x(q.reshape(S * Hh, D), q_sf.reshape(S * Hh, D // 128)).reshape(S, Hh, D)
+    K = dequant_w(kv[None], kv_sf[None])[0]                       # [N, D]
+    dots = np.einsum("shd,nd->shn", Q, K)                        # [S, Hh, N]
+    out = np.einsum("sh,shn->sn", weights.astype(np.float64), np.maximum(dots, 0.0))
+    j = np.arange(N)[None, :]
+    valid = (j >= np.maximum(ks, 0)[:, None]) & (j < np.minimum(ke, N)[:, None])
+    return np.where(valid, out, -np.inf)
