@@ -647,9 +647,107 @@ def run_gemm(args, name):
         "clocks": clk.summary(), "cpu_baseline": None}), flush=True)
 
 
+# ------------------------------------------------------- FP4 indexer (MQA logits)
+def run_indexer(args, name):
+    """The FP4 indexer: K timed replays of one captured call (key layout and
+    scale chunks rebuilt inside the call), L2 flushed before each, one JSON line."""
+    import numpy as np
+    import torch
+
+    import block_scaled_fp8_permute_b200 as moe
+    import oracle
+    import synth
+
+    wl = synth.INDEXER_WORKLOADS[name]
+    d = synth.make_indexer(wl.S, wl.Hh, wl.D, wl.N, wl.seed)
+    dev = "cuda:0"
+    t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(dev) for k, v in d.items()}
+    out = torch.empty((wl.S, wl.N), dtype=torch.float32, device=dev)
+    ws = moe.alloc_mqa_workspace(wl.S, wl.Hh, wl.D, wl.N, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        moe.moe_fp8_fp4_mqa_logits(t["q"], t["q_sf"], t["kv"], t["kv_sf"], t["weights"], t["ks"],
+                                   t["ke"], out, ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        call()
+    stream.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status(ws) == 0
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    with ClockSampler(0) as clk:
+        clk.wait_first()
+        clk.mark("start")
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            graph.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        clk.mark("end")
+    ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
+    del graph
+    S, Hh, D, N = wl.S, wl.Hh, wl.D, wl.N
+    algo_bytes = (S * Hh * (D + D // 32) + N * (D // 2 + D // 32) + S * Hh * 4 + S * 8
+                  + S * N * 4)
+    pk = _peaks()
+    tpeak, hpeak = 2.0 * pk["bf16"], pk["hbm"]
+    tflops = wl.flops / (ms * 1e-3) / 1e12
+    gbs = algo_bytes / (ms * 1e-3) / 1e9
+    if wl.flops / (tpeak * 1e12) >= algo_bytes / (hpeak * 1e9):
+        roof = {"bound": "tensor", "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s",
+                "peak_note": f"2 x bf16 burst {pk['bf16']} TFLOP/s ({pk['src']})"}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hpeak, "unit": "GB/s",
+                "peak_note": f"copy bandwidth {hpeak} GB/s ({pk['src']})"}
+    roof.update(frac=roof["achieved"] / roof["peak"], kernel="mqa_logits_kernel",
+                flops_per_launch=wl.flops, algorithmic_bytes_per_launch=algo_bytes, traffic=None)
+    cpu = None
+    if not args.no_cpu_baseline:
+        rows = np.arange(min(S, 8), dtype=np.int64)
+        sub = dict(d)
+        for k in ("q", "q_sf", "weights", "ks", "ke"):
+            sub[k] = np.ascontiguousarray(d[k][rows])
+        t0 = time.perf_counter()
+        oracle.mqa_logits(**sub)
+        sec = time.perf_counter() - t0
+        pairs = int(sum(max(0, min(int(sub["ke"][r]), N) - max(int(sub["ks"][r]), 0))
+                        for r in range(len(rows))))
+        cpu = {"value": 2.0 * Hh * D * pairs / sec / 1e12, "unit": "TFLOPS",
+               "cores": oracle.max_threads(), "kind": "oracle",
+               "sample": f"{len(rows)} query rows of {S} (all their keys), {sec:.1f} s"}
+    print(json.dumps({
+        "metric": "FP4-indexer MQA logits TFLOPS on 1 B200 (FP8 q x FP4 k, FP32 logits)",
+        "value": tflops, "unit": "TFLOPS", "gbs": gbs, "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3 x fp4_e2m1, fp32 accumulate, fp32 out",
+        "data": "synthetic",
+        "config": {"workload": f"{name}: S={S} Hh={Hh} D={D} N={N}, query i sees keys "
+                               f"[0, N - S + i + 1)", "l2": "flushed before every step",
+                   "step": "one call replayed as a CUDA graph (key layout rebuilt inside)"},
+        "roofline": roof,
+        "gpu_launches": 3 * K,  # key layout, query scale chunks, logits
+        "clocks": clk.summary(), "cpu_baseline": cpu}), flush=True)
+
+
 def main():
     args = _args()
     import synth
+    if args.workload in synth.INDEXER_WORKLOADS:
+        if int(os.environ.get("RANK", "0")) == 0 and args.impl == "ours":
+            run_indexer(args, args.workload)
+        return
     if args.workload in GEMM_SHAPES:
         if int(os.environ.get("RANK", "0")) == 0 and args.impl == "ours":
             run_gemm(args, args.workload)

@@ -72,6 +72,8 @@ _SIGS = {
     "moe_gemm_workspace_bytes": (_sz, [_i, _i, _i, _i]),
     "moe_gemm_fp8_fp4": (_i, [_i, _i, _i] + [_vp] * 6 + [_sz, _vp]),
     "moe_gemm_fp8_fp4_masked": (_i, [_i, _i, _i, _i] + [_vp] * 7 + [_sz, _vp]),
+    "moe_mqa_logits_workspace_bytes": (_sz, [_i, _i, _i, _i]),
+    "moe_fp8_fp4_mqa_logits": (_i, [_i, _i, _i, _i] + [_vp] * 7 + [_i, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -320,3 +322,29 @@ def alloc_gemm_workspace(G, M_max, N, K, device):
     import torch
     n = moe_gemm_workspace_bytes(G, M_max, N, K)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------ FP4 indexer
+def moe_mqa_logits_workspace_bytes(S: int, Hh: int, D: int, N: int) -> int:
+    return _lib.moe_mqa_logits_workspace_bytes(S, Hh, D, N)
+
+
+def moe_fp8_fp4_mqa_logits(q, q_sf, kv, kv_sf, weights, ks, ke, logits, workspace, clean=True,
+                           ws_bytes=None, stream=None):
+    """logits [S, N] (fp32, device) of FP8 queries q [S, Hh, D] against FP4
+    keys kv [N, D/2]; see include/moe.h for the layouts."""
+    S, Hh, D = q.shape
+    N = kv.shape[0]
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+    _check("moe_fp8_fp4_mqa_logits", _lib.moe_fp8_fp4_mqa_logits(
+        S, Hh, D, N, _ptr(q), _ptr(q_sf), _ptr(kv), _ptr(kv_sf), _ptr(weights), _ptr(ks),
+        _ptr(ke), 1 if clean else 0, _ptr(logits), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def alloc_mqa_workspace(S, Hh, D, N, device):
+    import torch
+    n = moe_mqa_logits_workspace_bytes(S, Hh, D, N)
+    if n == 0:
+        raise MoeError("moe_mqa_logits_workspace_bytes", 2)
+    return torch.empty(n, dtype=torch.uint8, device=device)

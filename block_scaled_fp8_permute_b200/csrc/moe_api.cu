@@ -17,7 +17,8 @@ cudaError_t launch_gemm_pair(int epi, const CUtensorMap& tmA, const CUtensorMap&
                              bool pdl, cudaStream_t stream);
 cudaError_t launch_requant_debug(const float* a, int rows, int cols, uint8_t* codes,
                                  uint8_t* sbytes, cudaStream_t stream);
-cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max, int narrow_max,
+cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int P_max, int swap_max,
+                        int narrow_max,
                         int* chunk, int* counts, int* offs, int* poffs, int* tile_expert,
                         int* mpair, int* norm_mtiles, int* swap_experts, int* narrow_mtiles,
                         int* row_of, int* src_of, int* hdr, bool pdl, cudaStream_t stream);
@@ -33,6 +34,15 @@ cudaError_t launch_transform(const uint8_t* w, const uint8_t* w_sf, int E, int N
 cudaError_t launch_gemm_prep(const int* masked_m, int G, int m_max, int mt_per_g, int* tile_expert,
                              int* norm_mtiles, int* hdr, const int32_t* a_sf, long long rows, int KG,
                              uint8_t* sf_chunks, cudaStream_t stream);
+
+cudaError_t launch_sf_chunks(const int32_t* a_sf, long long rows, int KG, uint8_t* sf_chunks,
+                             cudaStream_t stream);
+cudaError_t launch_kv_prep(const uint8_t* kv, const uint8_t* kv_sf, int N, int Np, int D,
+                           uint8_t* codes, uint8_t* chunks, cudaStream_t stream);
+cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, const uint8_t* sfa,
+                              const uint8_t* sfb, const float* w, const int* ks, const int* ke,
+                              float* out, int* hdr, int S, int Hh, int N, int KB, int clean,
+                              int grid, bool pdl, cudaStream_t stream);
 
 namespace {
 
@@ -281,6 +291,40 @@ moe_status gemm_run(int G, int M_max, int N, int K, const uint8_t* a, const int3
       launch_gemm(3, false, tmA, tmA, tmB, tmD, g, grid < 1 ? 1 : grid, g_pdl.load() != 0, s));
 }
 
+// FP4 indexer (MQA logits): shape rules and workspace (status header, keys in
+// the tile layout, key and query scale chunks)
+moe_status check_mqa(int S, int Hh, int D, int N) {
+  if (S < 0 || N < 0 || D <= 0 || Hh <= 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (Hh != 16 && Hh != 32 && Hh != 64 && Hh != 128) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (D % 128 || D > 1024) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)S * Hh > (1LL << 24) || N > (1 << 24) || (long long)S * N > (1LL << 34))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+struct MqaWs {
+  size_t hdr, codes, kchunks, qchunks, total;
+  int Np, n_groups;
+};
+MqaWs mqa_ws(int S, int Hh, int D, int N) {
+  MqaWs w{};
+  w.Np = (N + 127) / 128 * 128;
+  w.n_groups = (int)(((long long)S * Hh + 255) / 256);
+  const int KB = D / 128;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  w.hdr = take(kHdrWords * 4);
+  w.codes = take((size_t)KB * w.Np * 64);
+  w.kchunks = take((size_t)KB * (w.Np / 128) * kSfChunk);
+  w.qchunks = take((size_t)2 * w.n_groups * KB * kSfChunk);
+  w.total = off;
+  return w;
+}
+
 // staging area of moe_forward_host, after the regular workspace
 struct HostStage {
   size_t x, x_sf, idx, w, y, total;
@@ -403,7 +447,7 @@ moe_status moe_plan(const moe_shape* shape, const int32_t* topk_idx, void* works
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(ws.hdr(), 0, kHdrWords * 4, s);
   if (e == cudaSuccess)
-    e = launch_plan(topk_idx, ws.L.R, shape->E, ws.L.NCH, g_swap_max.load(),
+    e = launch_plan(topk_idx, ws.L.R, shape->E, ws.L.NCH, ws.L.P_max, g_swap_max.load(),
                     narrow_max_for(*shape), ws.chunk(), ws.counts(), ws.offs(), ws.poffs(),
                     ws.tile_expert(), ws.mpair(), ws.norm_mt(), ws.swap_e(), ws.narrow_mt(),
                     ws.row_of(), ws.src_of(), ws.hdr(), g_pdl.load() != 0, s);
@@ -714,6 +758,50 @@ moe_status moe_gemm_fp8_fp4_masked(int G, int M_max, int N, int K, const uint8_t
   if (!masked_m) return MOE_ERR_INVALID_ARG;
   return gemm_run(G, M_max, N, K, a, a_sf, masked_m, b_t, b_sf_t, d, workspace, ws_bytes,
                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t moe_mqa_logits_workspace_bytes(int S, int Hh, int D, int N) {
+  if (check_mqa(S, Hh, D, N) != MOE_OK) return 0;
+  return mqa_ws(S, Hh, D, N).total;
+}
+
+moe_status moe_fp8_fp4_mqa_logits(int S, int Hh, int D, int N, const uint8_t* q,
+                                  const int32_t* q_sf, const uint8_t* kv, const uint8_t* kv_sf,
+                                  const float* weights, const int32_t* ks, const int32_t* ke,
+                                  int clean, float* logits, void* workspace, size_t ws_bytes,
+                                  moe_stream_t stream) {
+  moe_status st = check_mqa(S, Hh, D, N);
+  if (st != MOE_OK) return st;
+  const MqaWs L = mqa_ws(S, Hh, D, N);
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (S == 0 || N == 0) return MOE_OK;
+  const void* p16[] = {q, kv, weights};
+  for (const void* p : p16)
+    if (!p || !aligned(p, 16)) return MOE_ERR_INVALID_ARG;
+  const void* p4[] = {q_sf, kv_sf, ks, ke, logits};
+  for (const void* p : p4)
+    if (!p || !aligned(p, 4)) return MOE_ERR_INVALID_ARG;
+  const int sms = device_sms();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  int* hdr = reinterpret_cast<int*>(base + L.hdr);
+  uint8_t* codes = base + L.codes;
+  uint8_t* kchunks = base + L.kchunks;
+  uint8_t* qchunks = base + L.qchunks;
+  const int KB = D / 128;
+  CUtensorMap tmK, tmQ;
+  if (!encode_wgt(&tmK, codes, 1, KB, L.Np, 128) || !encode_act(&tmQ, q, S * Hh, D, 256))
+    return MOE_ERR_CUDA;
+  cudaError_t e = cudaMemsetAsync(hdr, 0, kHdrWords * 4, s);
+  if (e == cudaSuccess) e = launch_kv_prep(kv, kv_sf, N, L.Np, D, codes, kchunks, s);
+  if (e == cudaSuccess) e = launch_sf_chunks(q_sf, (long long)S * Hh, KB, qchunks, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  const long long tiles = (long long)(L.Np / 128) * L.n_groups;
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  return cuda_status(launch_mqa_logits(tmK, tmQ, kchunks, qchunks, weights, ks, ke, logits, hdr, S,
+                                       Hh, N, KB, clean ? 1 : 0, grid, g_pdl.load() != 0, s));
 }
 
 moe_status moe_debug_requant(const float* a, int rows, int cols, uint8_t* codes, uint8_t* sbytes,

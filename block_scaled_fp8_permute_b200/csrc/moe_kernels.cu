@@ -24,16 +24,16 @@ __device__ __forceinline__ size_t sf_chunk_offset(int row, int kg, int G) {
 }
 
 // ------------------------------------------------------------------- plan
-// K1 (count + scan, one launch): every block histograms its chunk of
-// kPlanChunk consecutive flattened slots into chunk_counts[b][e]; the last
-// block to finish then turns the chunk histograms into per-chunk starting
-// ranks (exclusive, in place), expert counts, offsets, padded offsets, the
-// m-tile -> expert table, the m-tile pairs and m-tiles of normal-tiled
-// experts, the list of swapped-role experts (1 <= count <= swap_max), the
-// m-tiles of narrow-tiled experts (1 <= count <= narrow_max) and -1
-// for the padding rows of src_of.
+// K1 (count + scan, one launch): every block fills its share of src_of with
+// -1 (padding) and histograms its chunk of kPlanChunk consecutive flattened
+// slots into chunk_counts[b][e]; the last block to finish then turns the
+// chunk histograms into per-chunk starting ranks (exclusive, in place),
+// expert counts, offsets, padded offsets, the m-tile -> expert table, the
+// m-tile pairs and m-tiles of normal-tiled experts, the list of swapped-role
+// experts (1 <= count <= swap_max) and the m-tiles of narrow-tiled experts
+// (1 <= count <= narrow_max).
 __global__ void __launch_bounds__(1024) plan_count_scan_kernel(
-    const int32_t* __restrict__ idx, int R, int E, int NCH, int swap_max, int narrow_max,
+    const int32_t* __restrict__ idx, int R, int E, int NCH, int P_max, int swap_max, int narrow_max,
     int* __restrict__ chunk_counts, int* __restrict__ counts, int* __restrict__ offs,
     int* __restrict__ poffs, int* __restrict__ tile_expert, int* __restrict__ mpair,
     int* __restrict__ norm_mtiles, int* __restrict__ swap_experts, int* __restrict__ narrow_mtiles,
@@ -43,6 +43,11 @@ __global__ void __launch_bounds__(1024) plan_count_scan_kernel(
   __shared__ int last_block;
   const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) hist[e] = 0;
+  // every row starts as padding (-1); the scatter kernel that follows
+  // overwrites the rows that hold assignments.  Filled by all blocks, so no
+  // single block writes the padding of every expert.
+  for (int r = blockIdx.x * blockDim.x + tid; r < P_max; r += gridDim.x * blockDim.x)
+    src_of[r] = -1;
   __syncthreads();
   const int a = blockIdx.x * kPlanChunk + tid;
   if (a < R) {
@@ -143,7 +148,6 @@ __global__ void __launch_bounds__(1024) plan_count_scan_kernel(
       for (int i = 0; i < nm; ++i) norm_mtiles[pre[3] + i] = mt_first + i;
       if (swapped) swap_experts[pre[4]] = e;
       if (narrow) narrow_mtiles[pre[5]] = mt_first;
-      for (int r = pre[1] + c; r < pre[1] + pc; ++r) src_of[r] = -1;
     }
     __syncthreads();
     if (tid < NV) carry[tid] += warp_tot[tid][31];
@@ -331,6 +335,15 @@ __global__ void sf_chunks_kernel(const int32_t* __restrict__ a_sf, long long row
   }
 }
 
+cudaError_t launch_sf_chunks(const int32_t* a_sf, long long rows, int KG, uint8_t* sf_chunks,
+                             cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  long long grid = (rows * KG + 255) / 256;
+  if (grid > 148LL * 16) grid = 148LL * 16;
+  sf_chunks_kernel<<<(unsigned)grid, 256, 0, stream>>>(a_sf, rows, KG, sf_chunks);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm_prep(const int* masked_m, int G, int m_max, int mt_per_g, int* tile_expert,
                              int* norm_mtiles, int* hdr, const int32_t* a_sf, long long rows, int KG,
                              uint8_t* sf_chunks, cudaStream_t stream) {
@@ -391,7 +404,8 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max, int narrow_max,
+cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int P_max, int swap_max,
+                        int narrow_max,
                         int* chunk, int* counts, int* offs, int* poffs, int* tile_expert,
                         int* mpair, int* norm_mtiles, int* swap_experts, int* narrow_mtiles,
                         int* row_of, int* src_of, int* hdr, bool pdl, cudaStream_t stream) {
@@ -405,7 +419,7 @@ cudaError_t launch_plan(const int32_t* idx, int R, int E, int NCH, int swap_max,
     attr_set = true;
   }
   plan_count_scan_kernel<<<NCH > 0 ? NCH : 1, 1024, 0, stream>>>(
-      idx, R, E, NCH, swap_max, narrow_max, chunk, counts, offs, poffs, tile_expert, mpair,
+      idx, R, E, NCH, P_max, swap_max, narrow_max, chunk, counts, offs, poffs, tile_expert, mpair,
       norm_mtiles, swap_experts, narrow_mtiles, src_of, hdr);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || R == 0) return e;

@@ -327,6 +327,41 @@ moe_status moe_gemm_fp8_fp4_masked(int G, int M_max, int N, int K, const uint8_t
                                    const void* b_sf_t, uint16_t* d, void* workspace,
                                    size_t ws_bytes, moe_stream_t stream);
 
+/* ------------------------------------------------------ FP4 indexer (MQA) */
+/* MQA logits of the lightning indexer with FP8 queries and FP4 keys
+ * ("DeepSeek DeepGEMM 2026年4月重磅更新" section 5.1, the fp8_fp4_mqa_logits
+ * call: q, kv, per-head weights, per-query key ranges cu_seq_len_k_start /
+ * cu_seq_len_k_end, clean_logits; section 5.2, the logit of query i and
+ * key j).  The page's formula is garbled (a ReLU of a softmax); this library
+ * computes, for every query token i and key j with ks[i] <= j < ke[i]:
+ *   logits[i][j] = sum_h weights[i][h] * max(0, sum_d q[i][h][d] * k[j][d])
+ * with FP32 accumulation; entries outside the range are -inf when `clean`
+ * is non-zero and are not written otherwise.
+ *   q       uint8 [S, Hh, D]  E4M3 codes (the query heads of each token)
+ *   q_sf    int32 [S, Hh, D/128]  UE8M0 scales per 1x32 block along D, four
+ *                             per word as x_sf
+ *   kv      uint8 [N, D/2]    E2M1 codes, two per byte, low nibble = even d
+ *   kv_sf   uint8 [N, D/32]   UE8M0 per 1x32 block
+ *   weights fp32  [S, Hh]
+ *   ks, ke  int32 [S]         key range of each query (clamped to [0, N];
+ *                             an empty range gives a row of -inf)
+ *   logits  fp32  [S, N]      row-major
+ * Shapes: Hh in {16, 32, 64, 128}, D a multiple of 128 up to 1024, S, N >= 0,
+ * S * Hh <= 2^24, N <= 2^24.  Pointers are caller-owned device memory: q, kv
+ * and weights 16-byte aligned, the rest 4-byte aligned, the workspace
+ * 256-byte aligned with moe_mqa_logits_workspace_bytes() bytes (the keys in
+ * the tile layout and the scale chunks, rebuilt by every call from the
+ * canonical inputs).  Errors: MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_INVALID_ARG,
+ * MOE_ERR_WORKSPACE, MOE_ERR_CUDA; a device wait that expires is reported by
+ * moe_get_device_status(workspace).  Enqueued on `stream`; nothing is
+ * synchronised. */
+size_t moe_mqa_logits_workspace_bytes(int S, int Hh, int D, int N);
+moe_status moe_fp8_fp4_mqa_logits(int S, int Hh, int D, int N, const uint8_t* q,
+                                  const int32_t* q_sf, const uint8_t* kv, const uint8_t* kv_sf,
+                                  const float* weights, const int32_t* ks, const int32_t* ke,
+                                  int clean, float* logits, void* workspace, size_t ws_bytes,
+                                  moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -364,8 +364,9 @@ int orc_max_threads(void) {
  * Layouts: q u8 [S, Hh, D] E4M3; q_sf i32 [S, Hh, D/128] (byte j of word i =
  * scale of block 4i+j, as x_sf); kv u8 [N, D/2] E2M1 (low nibble = even d);
  * kv_sf u8 [N, D/32]; weights f32 [S, Hh]; ks, ke i32 [S]; logits f32 [S, N].
- * When mag is not NULL, mag[i][j] = sum_h |weights[i][h] * dot_h| (a bound
- * on the size of every term, used to scale the comparison tolerance). */
+ * When mag is not NULL, mag[i][j] = sum_h |weights[i][h]| * sum_d |q[i][h][d] * k[j][d]|
+ * (the size of every product that enters the logit: a comparison with a
+ * lower-precision computation scales its tolerance by it). */
 void orc_mqa_logits(int S, int Hh, int D, int N, const uint8_t* q, const int32_t* q_sf,
                     const uint8_t* kv, const uint8_t* kv_sf, const float* weights,
                     const int32_t* ks, const int32_t* ke, int clean, float* logits, double* mag,
@@ -394,11 +395,14 @@ void orc_mqa_logits(int S, int Hh, int D, int N, const uint8_t* q, const int32_t
       for (int d = 0; d < D; ++d) kd[d] = w_value(kv, kv_sf, N, D, 0, j, d);
       double acc = 0.0, m = 0.0;
       for (int h = 0; h < Hh; ++h) {
-        double s = 0.0;
-        for (int d = 0; d < D; ++d) s += qd[(size_t)h * D + d] * kd[d];
+        double s = 0.0, sa = 0.0;
+        for (int d = 0; d < D; ++d) {
+          s += qd[(size_t)h * D + d] * kd[d];
+          sa += fabs(qd[(size_t)h * D + d] * kd[d]);
+        }
         double w = (double)weights[(size_t)i * Hh + h];
         if (s > 0.0) acc += w * s;
-        m += fabs(w * s);
+        m += fabs(w) * sa;
       }
       *out = (float)acc;
       if (mag) mag[(size_t)i * N + j] = m;

@@ -149,3 +149,50 @@ def workload(name: str) -> Workload:
         base, t = name.split("@T")
         return WORKLOADS[base].with_tokens(int(t))
     return WORKLOADS[name]
+
+
+# ------------------------------------------------------------ FP4 indexer
+@dataclasses.dataclass(frozen=True)
+class IndexerWorkload:
+    """MQA-logit workload of the FP4 indexer: S query tokens with Hh heads of
+    dimension D against N keys; query i sees keys [0, N - S + i + 1) (the
+    keys already cached plus the new tokens up to itself)."""
+    name: str
+    S: int
+    Hh: int
+    D: int
+    N: int
+    seed: int = 0
+
+    @property
+    def pairs(self) -> int:
+        """(query, key) pairs inside the ranges."""
+        return sum(self.N - self.S + i + 1 for i in range(self.S))
+
+    @property
+    def flops(self) -> float:
+        """2 * Hh * D per scored pair (the dot products; the weighted ReLU sum is not counted)."""
+        return 2.0 * self.Hh * self.D * self.pairs
+
+
+INDEXER_WORKLOADS = {
+    # prefill: 4096 new tokens over an 8192-token context, 64 index heads of dimension 128
+    "indexer": IndexerWorkload("indexer", 4096, 64, 128, 8192),
+    # decode with 4 multi-token-prediction tokens over a 65536-token context
+    "indexer-decode": IndexerWorkload("indexer-decode", 4, 64, 128, 65536),
+}
+
+
+def make_indexer(S: int, Hh: int, D: int, N: int, seed: int = 0):
+    """q u8 [S, Hh, D] E4M3 (+ q_sf i32 [S, Hh, D/128]) from the activation
+    generator, kv u8 [N, D/2] E2M1 (+ kv_sf u8 [N, D/32]) from the weight
+    generator (stream 6, std 1), weights f32 [S, Hh] ~ N(0, 1/Hh) and the
+    prefix ranges ks = 0, ke = N - S + i + 1 (clamped to [0, N])."""
+    q, q_sf = make_x(S * Hh, D, seed)
+    kv, kv_sf = make_w(1, N, D, 6, seed, std=1.0)
+    rng = np.random.default_rng(seed + 1000)
+    w = (rng.standard_normal((S, Hh)) / math.sqrt(Hh)).astype(np.float32)
+    ke = np.clip(N - S + 1 + np.arange(S), 0, N).astype(np.int32)
+    ks = np.zeros(S, np.int32)
+    return dict(q=q.reshape(S, Hh, D), q_sf=q_sf.reshape(S, Hh, D // 128), kv=kv[0],
+                kv_sf=kv_sf[0], weights=w, ks=ks, ke=ke)
