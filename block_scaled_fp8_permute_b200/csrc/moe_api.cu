@@ -39,10 +39,14 @@ cudaError_t launch_sf_chunks(const int32_t* a_sf, long long rows, int KG, uint8_
                              cudaStream_t stream);
 cudaError_t launch_kv_prep(const uint8_t* kv, const uint8_t* kv_sf, int N, int Np, int D,
                            uint8_t* codes, uint8_t* chunks, cudaStream_t stream);
+int mqa_tokens_per_tile(int Hh);
+size_t mqa_qsf_bytes_per_group(int D);
+cudaError_t launch_q_sf_prep(const int32_t* q_sf, long long rows, int D, int Hh, uint8_t* out,
+                             cudaStream_t stream);
 cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, const uint8_t* sfa,
                               const uint8_t* sfb, const float* w, const int* ks, const int* ke,
-                              float* out, int* hdr, int S, int Hh, int N, int KB, int clean,
-                              int grid, bool pdl, cudaStream_t stream);
+                              float* out, int* hdr, uint8_t* act, int S, int Hh, int N, int KB,
+                              int clean, int grid, bool pdl, cudaStream_t stream);
 
 namespace {
 
@@ -303,13 +307,13 @@ moe_status check_mqa(int S, int Hh, int D, int N) {
 }
 
 struct MqaWs {
-  size_t hdr, codes, kchunks, qchunks, total;
+  size_t hdr, codes, kchunks, qchunks, act, total;
   int Np, n_groups;
 };
 MqaWs mqa_ws(int S, int Hh, int D, int N) {
   MqaWs w{};
   w.Np = (N + 127) / 128 * 128;
-  w.n_groups = (int)(((long long)S * Hh + 255) / 256);
+  w.n_groups = (S + mqa_tokens_per_tile(Hh) - 1) / mqa_tokens_per_tile(Hh);
   const int KB = D / 128;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -320,7 +324,8 @@ MqaWs mqa_ws(int S, int Hh, int D, int N) {
   w.hdr = take(kHdrWords * 4);
   w.codes = take((size_t)KB * w.Np * 64);
   w.kchunks = take((size_t)KB * (w.Np / 128) * kSfChunk);
-  w.qchunks = take((size_t)2 * w.n_groups * KB * kSfChunk);
+  w.qchunks = take((size_t)w.n_groups * mqa_qsf_bytes_per_group(D));
+  w.act = take((size_t)w.n_groups * (w.Np / 128));
   w.total = off;
   return w;
 }
@@ -792,16 +797,18 @@ moe_status moe_fp8_fp4_mqa_logits(int S, int Hh, int D, int N, const uint8_t* q,
   uint8_t* qchunks = base + L.qchunks;
   const int KB = D / 128;
   CUtensorMap tmK, tmQ;
-  if (!encode_wgt(&tmK, codes, 1, KB, L.Np, 128) || !encode_act(&tmQ, q, S * Hh, D, 256))
+  if (!encode_wgt(&tmK, codes, 1, KB, L.Np, 128) ||
+      !encode_act(&tmQ, q, S * Hh, D, mqa_tokens_per_tile(Hh) * Hh))
     return MOE_ERR_CUDA;
   cudaError_t e = cudaMemsetAsync(hdr, 0, kHdrWords * 4, s);
   if (e == cudaSuccess) e = launch_kv_prep(kv, kv_sf, N, L.Np, D, codes, kchunks, s);
-  if (e == cudaSuccess) e = launch_sf_chunks(q_sf, (long long)S * Hh, KB, qchunks, s);
+  if (e == cudaSuccess) e = launch_q_sf_prep(q_sf, (long long)S * Hh, D, Hh, qchunks, s);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   const long long tiles = (long long)(L.Np / 128) * L.n_groups;
   const int grid = (int)(tiles < sms ? tiles : sms);
-  return cuda_status(launch_mqa_logits(tmK, tmQ, kchunks, qchunks, weights, ks, ke, logits, hdr, S,
-                                       Hh, N, KB, clean ? 1 : 0, grid, g_pdl.load() != 0, s));
+  return cuda_status(launch_mqa_logits(tmK, tmQ, kchunks, qchunks, weights, ks, ke, logits, hdr,
+                                       base + L.act, S, Hh, N, KB, clean ? 1 : 0, grid,
+                                       g_pdl.load() != 0, s));
 }
 
 moe_status moe_debug_requant(const float* a, int rows, int cols, uint8_t* codes, uint8_t* sbytes,

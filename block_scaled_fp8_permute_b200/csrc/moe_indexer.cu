@@ -8,17 +8,20 @@
 // q: FP8 E4M3 [S, Hh, D], k: FP4 E2M1 [N, D], both with one UE8M0 scale per
 // 1x32 block along D; FP32 accumulation and output.
 //
-// Tiling.  The keys sit on the MMA's M side (128 keys per tile) and the
-// queries' (token, head) rows on its N side (256 rows = 256/Hh tokens), so
-// every epilogue thread owns one key and holds all heads of its tokens in
-// its accumulator columns: the head-weighted ReLU sum is a per-thread loop,
-// no cross-lane reduction.  One CTA per SM, persistent, 320 threads:
+// Tiling.  The keys sit on the MMA's M side (128 keys per tile) and a group
+// of query tokens' (token, head) rows on its N side (kTok tokens, kN =
+// kTok * Hh <= 192 rows), so every epilogue thread owns one key and holds all
+// heads of its tokens in its accumulator columns: the head-weighted ReLU sum
+// is a per-thread loop, no cross-lane reduction.  That sum costs about as
+// much as the tile's MMAs, so the accumulator is double-buffered in TMEM
+// (two 192-column buffers) and the MMAs of one tile run while the epilogue
+// reduces the previous one.  One CTA per SM, persistent, 320 threads:
 //   warp 0     TMA producer: key tile 128 x 128 (E2M1, unpacked by the TMA),
-//              query tile 256 x 128 (E4M3), their scale chunks; 4-stage ring
+//              query tile kN x 128 (E4M3), their scale chunks; 4-stage ring
 //   warp 1     TMEM allocator and MMA issuer (tcgen05.mma kind::mxf8f6f4,
-//              A = keys E2M1, B = queries E4M3, M=128, N=256, K=32)
-//   warps 2-9  epilogue: two warps per 32-lane TMEM subpartition, one column
-//              half (128 columns = 128/Hh tokens) each
+//              A = keys E2M1, B = queries E4M3, M=128, N=kN, K=32)
+//   warps 2-13 epilogue: three warps per 32-lane TMEM subpartition, the
+//              group's tokens split between them
 // Tiles whose keys lie outside every token's [ks, ke) skip the loads and the
 // MMAs; the epilogue only writes their -inf entries.
 #include "moe_device.cuh"
@@ -29,49 +32,76 @@ namespace moe {
 namespace {
 
 constexpr int kIdxStages = 4;
-constexpr int kIdxSmemA = 128 * 128;                 // keys, one byte per E2M1 element
-constexpr int kIdxSmemB = 256 * 128;                 // queries, E4M3
-constexpr int kIdxTxA = 128 * 128 / 2;               // bytes the TMA moves for the packed keys
-constexpr int kIdxEpiWarps = 8;
+constexpr int kIdxSmemA = 128 * 128;   // keys, one byte per E2M1 element
+constexpr int kIdxSmemB = 192 * 128;   // queries (up to 192 rows), E4M3
+constexpr int kIdxSmemSFB = 2 * kSfChunk;
+constexpr int kIdxTxA = 128 * 128 / 2; // bytes the TMA moves for the packed keys
+constexpr int kIdxEpiWarps = 12;  // three per 32-lane TMEM subpartition
 constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
 constexpr uint32_t kIdxTmemCols = 512;
-constexpr uint32_t kIdxSfCol = 256;
-constexpr size_t kIdxSmemBytes =
-    (size_t)kIdxStages * (kIdxSmemA + kIdxSmemB + kSfChunk + 2 * kSfChunk) + 256;
+constexpr uint32_t kIdxAccStride = 256;  // accumulator buffer b at column 256 b
+constexpr uint32_t kIdxSfCol = 448;      // scale buffers: SFA at +16b (4 cols), SFB at +16b+4 (8)
+// stage ring, then two weight slots (one per accumulator buffer: the group's
+// kN weights, 768 bytes), then barriers
+constexpr size_t kIdxSmemStage = (size_t)kIdxStages * (kIdxSmemA + kIdxSmemB + kSfChunk + kIdxSmemSFB);
+constexpr int kIdxWSlot = 1024;
+constexpr size_t kIdxSmemBytes = kIdxSmemStage + 2 * kIdxWSlot + 256;
 static_assert(kIdxSmemBytes <= 232448, "shared memory per CTA");
+static_assert(kIdxSmemA % 1024 == 0 && kIdxSmemB % 1024 == 0, "swizzled stage alignment");
+
+// tokens per tile for Hh heads: kN = kTok * Hh query rows on the MMA's N side
+__host__ __device__ constexpr int idx_tokens(int Hh) { return Hh >= 128 ? 1 : 192 / Hh; }
 
 struct IdxArgs {
   const uint8_t* sfa;    // key scale chunks [KB][ceil(N/128)][512]
-  const uint8_t* sfb;    // query scale chunks [ceil(S*Hh/128)][KB][512]
+  const uint8_t* sfb;    // query scale chunks [group][KB][2][512]
   const float* w;        // [S, Hh]
   const int* ks;         // [S]
   const int* ke;         // [S]
   float* out;            // [S, N]
   int* hdr;              // status header
+  const uint8_t* act;    // [n_groups * n_tiles_k]: 1 when some token of the group sees a key of the tile
   int S, Hh, N, KB, clean;
   int n_tiles_k;         // ceil(N / 128)
-  int n_groups;          // ceil(S / (256 / Hh))
+  int n_groups;          // ceil(S / tokens per tile)
 };
 
 // Does any token of query group g see a key of key tile kt?  (Decided the
 // same way by every role of the CTA.)
+template <int kTok>
 __device__ __forceinline__ bool tile_active(const IdxArgs& a, int kt, int g) {
-  const int tpg = 256 / a.Hh;
   const int j0 = kt * 128, j1 = min(j0 + 128, a.N);
-  for (int t = 0; t < tpg; ++t) {
-    const int i = g * tpg + t;
+#pragma unroll 1
+  for (int t = 0; t < kTok; ++t) {
+    const int i = g * kTok + t;
     if (i >= a.S) break;
-    const int lo = max(a.ks[i], 0), hi = min(a.ke[i], a.N);
+    const int lo = max(__ldg(a.ks + i), 0), hi = min(__ldg(a.ke + i), a.N);
     if (lo < j1 && hi > j0 && lo < hi) return true;
   }
   return false;
 }
 
-template <int kHh>  // heads per query token (divides 128)
+// Columns [c0, c0 + kHh) of this warp's 32 TMEM lanes -> registers.
+template <int kHh>
+__device__ __forceinline__ void load_head_cols(uint32_t taddr, uint32_t (&v)[kHh]) {
+  using namespace ptx;
+  if constexpr (kHh == 16) {
+    tmem_ld_32x32b_x16(taddr, v);
+  } else {
+#pragma unroll
+    for (int c = 0; c < kHh / 32; ++c)
+      tmem_ld_32x32b_x32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+  }
+}
+
+template <int kHh>  // heads per query token (16, 32, 64 or 128)
 __global__ void __launch_bounds__(kIdxThreads, 1)
     mqa_logits_kernel(const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmQ, const IdxArgs args) {
   using namespace ptx;
+  constexpr int kTok = idx_tokens(kHh);
+  constexpr int kN = kTok * kHh;
+  static_assert(kN % 16 == 0 && kN <= 192, "MMA N");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {  // the swizzled layout needs it; no work done yet
     if (threadIdx.x == 0) set_status(args.hdr, MOE_ERR_CUDA);
@@ -81,11 +111,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint8_t* sB = sA + kIdxStages * kIdxSmemA;
   uint8_t* sSFA = sB + kIdxStages * kIdxSmemB;
   uint8_t* sSFB = sSFA + kIdxStages * kSfChunk;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + kIdxStages * 2 * kSfChunk);
+  float* wslot = reinterpret_cast<float*>(smem_raw + kIdxSmemStage);  // [2][kIdxWSlot / 4]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + kIdxSmemStage + 2 * kIdxWSlot);
   uint64_t* empty = full + kIdxStages;
-  uint64_t* acc_full = empty + kIdxStages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
+  uint64_t* acc_full = empty + kIdxStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint64_t* w_full = acc_empty + 2;         // [2] weight slot b loaded
+  uint64_t* w_empty = w_full + 2;           // [2] weight slot b read by every epilogue warp
+  uint64_t* drain = w_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -95,8 +128,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kIdxEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kIdxEpiWarps);
+      mbar_init(&w_full[b], 1);
+      mbar_init(&w_empty[b], kIdxEpiWarps);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -118,16 +155,23 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   const int KB = args.KB;
   const int num_tiles = args.n_tiles_k * args.n_groups;
   uint32_t issued_mask = 0, last_phase = 0;
+  uint32_t w_issued = 0, w_phase = 0;  // weight slots loaded (producer lane), for the failure path
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t it = 0;
+      int tp = 0;  // active tiles so far
       bool ok = true;
+      const uint32_t tx = kIdxTxA + kN * 128 + kSfChunk + kIdxSmemSFB;
+      bool act = blockIdx.x < num_tiles && args.act[blockIdx.x];
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int nt = tile + gridDim.x;
+        const bool nact = nt < num_tiles && args.act[nt];  // loaded while this tile is issued
+        const bool cur = act;
+        act = nact;
+        if (!cur) continue;
         const int g = tile / args.n_tiles_k, kt = tile - g * args.n_tiles_k;
-        if (!tile_active(args, kt, g)) continue;
-        const uint32_t tx = kIdxTxA + kIdxSmemB + 3 * kSfChunk;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % kIdxStages;
           const uint32_t ph = (it / kIdxStages) & 1;
@@ -139,17 +183,31 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           }
           mbar_arrive_expect_tx(&full[s], tx);
           tma_load_3d(sA + s * kIdxSmemA, &tmK, &full[s], 0, kt * 128, kb);
-          tma_load_2d(sB + s * kIdxSmemB, &tmQ, &full[s], kb * 128, g * 256);
+          tma_load_2d(sB + s * kIdxSmemB, &tmQ, &full[s], kb * 128, g * kN);
           bulk_load(sSFA + s * kSfChunk,
                     args.sfa + ((size_t)kb * args.n_tiles_k + kt) * kSfChunk, kSfChunk, &full[s]);
-          // the group's 256 query rows are two 128-row chunks: [chunk][KB][512]
-          bulk_load(sSFB + s * 2 * kSfChunk,
-                    args.sfb + ((size_t)(2 * g) * KB + kb) * kSfChunk, kSfChunk, &full[s]);
-          bulk_load(sSFB + s * 2 * kSfChunk + kSfChunk,
-                    args.sfb + ((size_t)(2 * g + 1) * KB + kb) * kSfChunk, kSfChunk, &full[s]);
+          bulk_load(sSFB + s * kIdxSmemSFB, args.sfb + ((size_t)g * KB + kb) * kIdxSmemSFB,
+                    kIdxSmemSFB, &full[s]);
           issued_mask |= 1u << s;
           last_phase = (last_phase & ~(1u << s)) | (ph << s);
         }
+        if (!ok) break;
+        // the group's weights into the slot of this tile's accumulator buffer
+        // (rows of tokens past S are not read: the slot keeps stale values there)
+        const int b = tp & 1;
+        if (!mbar_wait_or_abort(&w_empty[b], ((tp >> 1) & 1) ^ 1, 2 * kWaitLimitNs, abort_flag)) {
+          if (!*abort_flag) record_timeout(args.hdr, 111);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const int ntok = min(kTok, args.S - g * kTok);
+        const uint32_t wbytes = (uint32_t)(ntok * kHh * 4);
+        mbar_arrive_expect_tx(&w_full[b], wbytes);
+        bulk_load(wslot + b * (kIdxWSlot / 4), args.w + (size_t)g * kN, wbytes, &w_full[b]);
+        w_issued |= 1u << b;
+        w_phase = (w_phase & ~(1u << b)) | ((uint32_t)((tp >> 1) & 1) << b);
+        ++tp;
       }
     }
   } else if (warp == 1) {
@@ -158,17 +216,24 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       uint32_t it = 0;
       int ta = 0;  // active tiles so far
       bool issued_any = false, ok = true;
-      const uint32_t idesc0 = idesc_mxf8f6f4(/*A E2M1*/ 5, /*B E4M3*/ 0, 128, 256);
+      const uint32_t idesc0 = idesc_mxf8f6f4(/*A E2M1*/ 5, /*B E4M3*/ 0, 128, kN);
       const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA)), b_desc0 = sdesc_sw128(smem_u32(sB));
       const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
+      bool act = blockIdx.x < num_tiles && args.act[blockIdx.x];
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int g = tile / args.n_tiles_k, kt = tile - g * args.n_tiles_k;
-        if (!tile_active(args, kt, g)) continue;
-        if (!mbar_wait_or_abort(acc_empty, (ta & 1) ^ 1, 2 * kWaitLimitNs, abort_flag)) {
+        const int nt = tile + gridDim.x;
+        const bool nact = nt < num_tiles && args.act[nt];  // loaded while this tile is issued
+        const bool cur = act;
+        act = nact;
+        if (!cur) continue;
+        const int b = ta & 1;
+        if (!mbar_wait_or_abort(&acc_empty[b], ((ta >> 1) & 1) ^ 1, 2 * kWaitLimitNs,
+                                abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t acc = tmem + kIdxAccStride * (uint32_t)b;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % kIdxStages;
           const uint32_t ph = (it / kIdxStages) & 1;
@@ -180,14 +245,16 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           const uint32_t sfa_t = tmem + kIdxSfCol + 16u * (it & 1u);
           const uint32_t sfb_t = sfa_t + 4u;
           tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + (uint64_t)((s * kSfChunk) >> 4));
-          tc_cp_32x128b_warpx4(sfb_t, sfb_desc0 + (uint64_t)((s * 2 * kSfChunk) >> 4));
-          tc_cp_32x128b_warpx4(sfb_t + 4u, sfb_desc0 + (uint64_t)((s * 2 * kSfChunk + kSfChunk) >> 4));
+          tc_cp_32x128b_warpx4(sfb_t, sfb_desc0 + (uint64_t)((s * kIdxSmemSFB) >> 4));
+          if (kN > 128)
+            tc_cp_32x128b_warpx4(sfb_t + 4u,
+                                 sfb_desc0 + (uint64_t)((s * kIdxSmemSFB + kSfChunk) >> 4));
           const uint64_t adesc = a_desc0 + (uint64_t)((s * kIdxSmemA) >> 4);
           const uint64_t bdesc = b_desc0 + (uint64_t)((s * kIdxSmemB) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t id = idesc_with_sf_id(idesc0, kk, kk);
-            mma_mxf8f6f4(tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id,
+            mma_mxf8f6f4(acc, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id,
                          (kb | kk) != 0 ? 1u : 0u, sfa_t | ((uint32_t)kk << 30),
                          sfb_t | ((uint32_t)kk << 30));
           }
@@ -195,7 +262,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           tc_commit(&empty[s]);
         }
         if (!ok) break;
-        tc_commit(acc_full);
+        tc_commit(&acc_full[b]);
         ++ta;
       }
       if (!ok) {
@@ -209,21 +276,35 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;        // 0..7
-    const int q = warp & 3;         // TMEM lane subpartition this warp can read
-    const int h = ew >> 2;          // column half: columns [128h, 128h + 128)
-    const int r = q * 32 + lane;    // key within the tile
+    const int ew = warp - 2;          // 0..11
+    const int q = warp & 3;           // TMEM lane subpartition this warp can read
+    const int h = ew >> 2;            // which of the group's tokens: t = h, h + 3, ...
+    const int r = q * 32 + lane;      // key within the tile
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-    constexpr int tpg = 256 / kHh, tph = 128 / kHh;  // tokens per group / per column half
+    constexpr int kMine = (kTok + 2) / 3;
     int ta = 0;
+    bool act_next = blockIdx.x < num_tiles && args.act[blockIdx.x];
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int g = tile / args.n_tiles_k, kt = tile - g * args.n_tiles_k;
       const int j = kt * 128 + r;
-      const bool active = tile_active(args, kt, g);
-      uint32_t v[4][32];
+      const bool active = act_next;
+      act_next = tile + (int)gridDim.x < num_tiles && args.act[tile + gridDim.x];
+      // key ranges of this warp's tokens (loaded before the waits)
+      int lo[kMine], hi[kMine];
+#pragma unroll
+      for (int m = 0; m < kMine; ++m) {
+        const int i = g * kTok + h + 3 * m;
+        const bool tok = h + 3 * m < kTok && i < args.S;
+        lo[m] = tok ? max(__ldg(args.ks + i), 0) : 0;
+        hi[m] = tok ? min(__ldg(args.ke + i), args.N) : 0;
+      }
+      const int b = ta & 1;
+      bool use = false;  // this tile's accumulator (and weight slot) is read
       if (active) {
-        const bool ready =
-            __all_sync(0xffffffffu, mbar_wait_or_abort(acc_full, ta & 1, 2 * kWaitLimitNs, abort_flag));
+        const uint32_t par = (ta >> 1) & 1;
+        const bool ready = __all_sync(0xffffffffu,
+                                      mbar_wait_or_abort(&acc_full[b], par, 2 * kWaitLimitNs, abort_flag) &&
+                                          mbar_wait_or_abort(&w_full[b], par, 2 * kWaitLimitNs, abort_flag));
         if (!ready) {
           if (lane == 0) {
             if (!*abort_flag) record_timeout(args.hdr, 130);
@@ -232,40 +313,66 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(trow + 128 * h + 32 * c, v[c]);
-        tc_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty);
-        ++ta;
+        use = true;
       }
-      // this thread's tokens: tph of them, kHh accumulator columns each
+      const float* w_s = wslot + b * (kIdxWSlot / 4);
+      // this warp's tokens t = h + 3m, in column chunks of at most 64: every
+      // TMEM load of a chunk first, one wait, then the weighted ReLU sums on
+      // eight independent accumulator chains
+      constexpr int kC = kHh > 64 ? 64 : kHh;  // columns per chunk
+      float acc[kMine][8];
 #pragma unroll
-      for (int t = 0; t < tph; ++t) {
-        const int i = g * tpg + h * tph + t;
-        if (i < args.S && j < args.N) {
-          const int lo = max(args.ks[i], 0), hi = min(args.ke[i], args.N);
-          float* dst = args.out + (size_t)i * args.N + j;
-          if (!active || j < lo || j >= hi) {
-            if (args.clean) *dst = -INFINITY;
-          } else {
-            const float4* wi = reinterpret_cast<const float4*>(args.w + (size_t)i * kHh);
-            float acc = 0.0f;
+      for (int m = 0; m < kMine; ++m)
 #pragma unroll
-            for (int h4 = 0; h4 < kHh / 4; ++h4) {
-              const float4 w4 = __ldg(wi + h4);
-              const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+        for (int u = 0; u < 8; ++u) acc[m][u] = 0.0f;
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int col = t * kHh + 4 * h4 + u;  // 0..127 inside the half
-                acc = fmaf(wv[u], fmaxf(__uint_as_float(v[col >> 5][col & 31]), 0.0f), acc);
+      for (int c0 = 0; c0 < kHh; c0 += kC) {
+        uint32_t v[kMine][kC];
+        if (use) {  // warp-uniform: the TMEM loads are collective
+#pragma unroll
+          for (int m = 0; m < kMine; ++m)
+            if (h + 3 * m < kTok)
+              load_head_cols<kC>(trow + kIdxAccStride * (uint32_t)b +
+                                     (uint32_t)((h + 3 * m) * kHh + c0), v[m]);
+          tc_wait_ld();
+#pragma unroll
+          for (int m = 0; m < kMine; ++m) {
+            const int t = h + 3 * m;
+            if (t < kTok) {
+              const float4* wt = reinterpret_cast<const float4*>(w_s + t * kHh + c0);
+#pragma unroll
+              for (int h4 = 0; h4 < kC / 4; ++h4) {
+                const float4 w4 = wt[h4];
+                const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  acc[m][(4 * h4 + u) & 7] = fmaf(wv[u], fmaxf(__uint_as_float(v[m][4 * h4 + u]), 0.0f),
+                                                  acc[m][(4 * h4 + u) & 7]);
               }
             }
-            *dst = acc;
           }
         }
       }
+      if (use) {  // accumulator and weights are in registers: release both
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&acc_empty[b]);
+          mbar_arrive(&w_empty[b]);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < kMine; ++m) {
+        const int t = h + 3 * m;
+        const int i = g * kTok + t;
+        const bool here = t < kTok && i < args.S && j < args.N;  // an entry of the output
+        const bool scored = use && here && j >= lo[m] && j < hi[m];
+        const float logit = scored ? ((acc[m][0] + acc[m][1]) + (acc[m][2] + acc[m][3])) +
+                                         ((acc[m][4] + acc[m][5]) + (acc[m][6] + acc[m][7]))
+                                   : -INFINITY;
+        if (scored || (here && args.clean)) args.out[(size_t)i * args.N + j] = logit;
+      }
+      if (active) ++ta;
     }
   }
 
@@ -276,11 +383,25 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // copies issued that nobody consumed land before the CTA's memory goes away
     for (int s = 0; s < kIdxStages; ++s)
       if (issued_mask & (1u << s)) (void)mbar_wait(&full[s], (last_phase >> s) & 1);
+    for (int b = 0; b < 2; ++b)
+      if (w_issued & (1u << b)) (void)mbar_wait(&w_full[b], (w_phase >> b) & 1);
   }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kIdxTmemCols);
+  }
+}
+
+// act[g * n_tiles_k + kt] = 1 when some token of query group g sees a key
+// of key tile kt.  One thread per tile.
+template <int kTok>
+__global__ void tile_activity_kernel(IdxArgs a, uint8_t* __restrict__ act) {
+  const long long total = (long long)a.n_groups * a.n_tiles_k;
+  for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total;
+       x += (long long)gridDim.x * blockDim.x) {
+    const int g = (int)(x / a.n_tiles_k), kt = (int)(x - (long long)g * a.n_tiles_k);
+    act[x] = tile_active<kTok>(a, kt, g) ? 1 : 0;
   }
 }
 
@@ -313,7 +434,30 @@ __global__ void kv_prep_kernel(const uint8_t* __restrict__ kv, const uint8_t* __
   }
 }
 
+// Query scales into per-group chunk pairs [group][KB][2][512 B]: query row r
+// (token * Hh + head) belongs to group r / kN, row rr = r % kN of it; chunk
+// rr / 128 of the pair, byte (rr%32)*16 + ((rr%128)/32)*4 + j.  Rows of the
+// pair past kN (or past the last token) stay whatever they were: their MMA
+// columns are never read.  One thread per (row, K-block).
+__global__ void q_sf_prep_kernel(const int32_t* __restrict__ q_sf, long long rows, int KB, int kN,
+                                 uint8_t* __restrict__ out) {
+  const long long total = rows * KB;
+  for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total;
+       x += (long long)gridDim.x * blockDim.x) {
+    const long long r = x / KB;
+    const int kb = (int)(x - r * KB);
+    const long long g = r / kN;
+    const int rr = (int)(r - g * kN);
+    uint8_t* dst = out + ((size_t)g * KB + kb) * kIdxSmemSFB + (rr >> 7) * kSfChunk;
+    const int r7 = rr & 127;
+    *reinterpret_cast<int32_t*>(dst + (r7 & 31) * 16 + (r7 >> 5) * 4) = q_sf[x];
+  }
+}
+
 }  // namespace
+
+int mqa_tokens_per_tile(int Hh) { return idx_tokens(Hh); }
+size_t mqa_qsf_bytes_per_group(int D) { return (size_t)(D / 128) * kIdxSmemSFB; }
 
 cudaError_t launch_kv_prep(const uint8_t* kv, const uint8_t* kv_sf, int N, int Np, int D,
                            uint8_t* codes, uint8_t* chunks, cudaStream_t stream) {
@@ -325,18 +469,32 @@ cudaError_t launch_kv_prep(const uint8_t* kv, const uint8_t* kv_sf, int N, int N
   return cudaGetLastError();
 }
 
+cudaError_t launch_q_sf_prep(const int32_t* q_sf, long long rows, int D, int Hh, uint8_t* out,
+                             cudaStream_t stream) {
+  const int KB = D / 128;
+  const long long total = rows * KB;
+  if (total == 0) return cudaSuccess;
+  long long grid = (total + 255) / 256;
+  if (grid > 148LL * 16) grid = 148LL * 16;
+  q_sf_prep_kernel<<<(unsigned)grid, 256, 0, stream>>>(q_sf, rows, KB,
+                                                       idx_tokens(Hh) * Hh, out);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, const uint8_t* sfa,
                               const uint8_t* sfb, const float* w, const int* ks, const int* ke,
-                              float* out, int* hdr, int S, int Hh, int N, int KB, int clean,
-                              int grid, bool pdl, cudaStream_t stream) {
+                              float* out, int* hdr, uint8_t* act, int S, int Hh, int N, int KB,
+                              int clean, int grid, bool pdl, cudaStream_t stream) {
   typedef void (*Fn)(CUtensorMap, CUtensorMap, IdxArgs);
+  typedef void (*ActFn)(IdxArgs, uint8_t*);
   Fn fn;
+  ActFn afn;
   int slot;
   switch (Hh) {
-    case 16: fn = mqa_logits_kernel<16>; slot = 0; break;
-    case 32: fn = mqa_logits_kernel<32>; slot = 1; break;
-    case 64: fn = mqa_logits_kernel<64>; slot = 2; break;
-    case 128: fn = mqa_logits_kernel<128>; slot = 3; break;
+    case 16: fn = mqa_logits_kernel<16>; afn = tile_activity_kernel<idx_tokens(16)>; slot = 0; break;
+    case 32: fn = mqa_logits_kernel<32>; afn = tile_activity_kernel<idx_tokens(32)>; slot = 1; break;
+    case 64: fn = mqa_logits_kernel<64>; afn = tile_activity_kernel<idx_tokens(64)>; slot = 2; break;
+    case 128: fn = mqa_logits_kernel<128>; afn = tile_activity_kernel<idx_tokens(128)>; slot = 3; break;
     default: return cudaErrorInvalidValue;
   }
   static bool attr_set[4] = {};
@@ -361,7 +519,17 @@ cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, co
   a.KB = KB;
   a.clean = clean;
   a.n_tiles_k = (N + 127) / 128;
-  a.n_groups = (S * Hh + 255) / 256;
+  a.n_groups = (S + idx_tokens(Hh) - 1) / idx_tokens(Hh);
+  a.act = act;
+  {
+    const long long tiles = (long long)a.n_tiles_k * a.n_groups;
+    long long agrid = (tiles + 255) / 256;
+    if (agrid > 148LL * 8) agrid = 148LL * 8;
+    if (agrid < 1) agrid = 1;
+    afn<<<(unsigned)agrid, 256, 0, stream>>>(a, act);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kIdxThreads);
