@@ -439,10 +439,29 @@ def measure(args, wl, inputs, dev, dist, weights=None, e2e=True):
             e1.synchronize()
             if i >= max(args.warmup, 3):
                 e2e_ms.append(e0.elapsed_time(e1))
-        rec["e2e_ms"] = statistics.mean(e2e_ms)
+        rec["e2e_serial_ms"] = statistics.mean(e2e_ms)
         rec["h2d"] = sum(t.numel() * t.element_size() for t in pin.values())
         rec["d2h"] = y_host.numel() * y_host.element_size()
         del ws_h
+        # the overlapped host-buffer call: K batches in one call, batch i + 1's
+        # inputs going up and batch i - 1's y coming down while batch i computes
+        ws_p = moe.alloc_workspace(shp, dev, host_variant="pipelined")
+        y2 = [y_host, torch.empty_like(y_host).pin_memory()]
+
+        def pipelined(n):
+            moe.moe_forward_host_pipelined(shp, [pin["x"]] * n, [pin["x_sf"]] * n,
+                                           [pin["topk_idx"]] * n, [pin["topk_w"]] * n, *lay.wt,
+                                           [y2[i & 1] for i in range(n)], ws_p)
+        flush.zero_()
+        pipelined(max(args.warmup, 3))
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pipelined(K)
+        e1.record(stream)
+        e1.synchronize()
+        rec["e2e_ms"] = e0.elapsed_time(e1) / K
+        del ws_p, y2
     del flush
     return rec, lay
 
@@ -483,7 +502,8 @@ def sub_record(args, wl, pk):
            "kernels_ms": rec["kernels_ms"], "clocks": rec["clocks"],
            "e2e": {"value": wl.flops / (rec["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
                    "ms_per_step": rec["e2e_ms"], "h2d_bytes_per_step": rec["h2d"],
-                   "d2h_bytes_per_step": rec["d2h"]},
+                   "d2h_bytes_per_step": rec["d2h"], "mode": "pipelined",
+                   "serial_ms_per_step": rec["e2e_serial_ms"]},
            "gpu_launches_per_step": _launches_per_step(wl)}
     if not args.no_cpu_baseline:
         out["cpu_baseline"] = _cpu_baseline(wl, inputs, args.sub_cpu_seconds)
@@ -505,6 +525,7 @@ def run_ours(args, wl, dist, rank, world, local_rank):
     rec, lay = measure(args, wl, inputs, dev, dist)
     ms = max_over_ranks(rec["ms"], dist, dev)
     e2e = max_over_ranks(rec["e2e_ms"], dist, dev)
+    e2e_serial = max_over_ranks(rec["e2e_serial_ms"], dist, dev)
     g1 = max_over_ranks(rec["kernels_ms"]["linear1"], dist, dev)
     del lay
     subs = {}
@@ -542,7 +563,11 @@ def run_ours(args, wl, dist, rank, world, local_rank):
         "step_roofline": step,
         "e2e": {"value": flops / (e2e * 1e-3) / 1e12, "unit": "TFLOPS",
                 "h2d_bytes_per_step": rec["h2d"], "d2h_bytes_per_step": rec["d2h"],
-                "ms_per_step": e2e},
+                "ms_per_step": e2e,
+                "mode": ("moe_forward_host_pipelined over the K steps (pinned host buffers; "
+                         "step i+1's inputs up and step i-1's y down while step i computes)"),
+                "serial_ms_per_step": e2e_serial,
+                "serial_note": "moe_forward_host, one synchronous call per step"},
         "gpu_launches": _launches_per_step(wl) * args.steps,
         "clocks": rec["clocks"],
         "cpu_baseline": cpu,

@@ -59,6 +59,9 @@ _SIGS = {
     "moe_forward": (_i, [_shp] + [_vp] * 9 + [_vp, _sz, _vp]),
     "moe_workspace_bytes_host": (_sz, [_shp]),
     "moe_forward_host": (_i, [_shp] + [_vp] * 9 + [_vp, _sz, _vp]),
+    "moe_workspace_bytes_host_pipelined": (_sz, [_shp]),
+    "moe_forward_host_pipelined": (_i, [_shp, _i] + [ctypes.POINTER(_vp)] * 4 + [_vp] * 4
+                                   + [ctypes.POINTER(_vp), _vp, _sz, _vp]),
     "moe_get_device_status": (_i, [_vp, _vp]),
     "moe_get_timeout_site": (_i, [_vp, _vp]),
     "moe_debug_set_fault": (None, [_i, ctypes.c_ulonglong]),
@@ -193,6 +196,30 @@ def moe_forward_host(shp, x, x_sf, topk_idx, topk_w, w1_t, w1_sf_t, w2_t, w2_sf_
         _stream(stream)))
 
 
+def moe_workspace_bytes_host_pipelined(shp: MoeShape) -> int:
+    return _lib.moe_workspace_bytes_host_pipelined(ctypes.byref(shp))
+
+
+def moe_forward_host_pipelined(shp, xs, x_sfs, topk_idxs, topk_ws, w1_t, w1_sf_t, w2_t, w2_sf_t,
+                               ys, workspace, ws_bytes=None, stream=None):
+    """len(xs) successive host-buffer forwards: xs, x_sfs, topk_idxs, topk_ws
+    and ys are equal-length lists of HOST buffers (pinned torch tensors or
+    numpy arrays), batch i reading the i-th of each and writing ys[i]."""
+    n = len(xs)
+    if not (len(x_sfs) == len(topk_idxs) == len(topk_ws) == len(ys) == n):
+        raise ValueError("moe_forward_host_pipelined: the buffer lists differ in length")
+    if ws_bytes is None:
+        ws_bytes = workspace.numel() * workspace.element_size()
+
+    def arr(bufs):
+        return (_vp * max(n, 1))(*[_ptr(b) for b in bufs])
+
+    _check("moe_forward_host_pipelined", _lib.moe_forward_host_pipelined(
+        ctypes.byref(shp), n, arr(xs), arr(x_sfs), arr(topk_idxs), arr(topk_ws), _ptr(w1_t),
+        _ptr(w1_sf_t), _ptr(w2_t), _ptr(w2_sf_t), arr(ys), _ptr(workspace), ws_bytes,
+        _stream(stream)))
+
+
 def moe_forward_noalloc(shp, x, x_sf, topk_idx, topk_w, w1_t, w1_sf_t, w2_t, w2_sf_t, y,
                         stream=None):
     """moe_plan + moe_forward on the library's own fixed 32 MiB workspace
@@ -303,8 +330,15 @@ def transform_weights(shp, w1, w1_sf, w2, w2_sf, stream=None):
 
 
 def alloc_workspace(shp, device, host_variant=False):
+    """host_variant: False (moe_plan / moe_forward), True (moe_forward_host) or
+    "pipelined" (moe_forward_host_pipelined)."""
     import torch
-    n = moe_workspace_bytes_host(shp) if host_variant else moe_workspace_bytes(shp)
+    if host_variant == "pipelined":
+        n = moe_workspace_bytes_host_pipelined(shp)
+    elif host_variant:
+        n = moe_workspace_bytes_host(shp)
+    else:
+        n = moe_workspace_bytes(shp)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
 
 

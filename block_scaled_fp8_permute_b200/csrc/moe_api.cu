@@ -665,6 +665,108 @@ moe_status moe_forward_host(const moe_shape* shape, const uint8_t* x_host,
   return cuda_status(e);
 }
 
+size_t moe_workspace_bytes_host_pipelined(const moe_shape* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  WsLayout L = ws_layout(*shape);
+  return host_stage(*shape, host_stage(*shape, L.total).total).total;
+}
+
+moe_status moe_forward_host_pipelined(const moe_shape* shape, int n_batches,
+                                      const uint8_t* const* x_host,
+                                      const int32_t* const* x_sf_host,
+                                      const int32_t* const* topk_idx_host,
+                                      const float* const* topk_w_host, const void* w1_t,
+                                      const void* w1_sf_t, const void* w2_t,
+                                      const void* w2_sf_t, uint16_t* const* y_host,
+                                      void* workspace, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (n_batches < 0) return MOE_ERR_INVALID_ARG;
+  const moe_shape sh = *shape;
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(sh);
+  const HostStage slot[2] = {host_stage(sh, L.total), host_stage(sh, host_stage(sh, L.total).total)};
+  if (ws_bytes < slot[1].total) return MOE_ERR_WORKSPACE;
+  if (sh.T == 0 || n_batches == 0) return MOE_OK;
+  if (!x_host || !x_sf_host || !topk_idx_host || !topk_w_host || !y_host)
+    return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_batches; ++i)
+    if (!x_host[i] || !x_sf_host[i] || !topk_idx_host[i] || !topk_w_host[i] || !y_host[i])
+      return MOE_ERR_INVALID_ARG;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t nx = (size_t)sh.T * sh.H, nsf = (size_t)sh.T * (sh.H / 128) * 4,
+               nk = (size_t)sh.T * sh.topk * 4, ny = (size_t)sh.T * sh.H * 2;
+
+  // Copy-in and copy-out run on streams of their own, so batch i + 1's inputs
+  // go up and batch i - 1's y comes down while batch i's kernels run on
+  // `stream`.  Staging slot i % 2 holds batch i; the events order its reuse.
+  cudaStream_t cin = nullptr, cout = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
+  cudaError_t e = cudaStreamCreateWithFlags(&cin, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&cout, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+  for (int b = 0; b < 2 && e == cudaSuccess; ++b) {
+    e = cudaEventCreateWithFlags(&ev_in[b], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_comp[b], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_out[b], cudaEventDisableTiming);
+  }
+  // both copy streams start after whatever the caller enqueued on `stream`
+  if (e == cudaSuccess) e = cudaEventRecord(ev_start, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cin, ev_start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cout, ev_start, 0);
+  st = cuda_status(e);
+  for (int i = 0; i < n_batches && st == MOE_OK; ++i) {
+    const int b = i & 1;
+    const HostStage& h = slot[b];
+    // slot b's inputs are overwritten once batch i - 2's kernels have read them
+    if (i >= 2) e = cudaStreamWaitEvent(cin, ev_comp[b], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(base + h.x, x_host[i], nx, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(base + h.x_sf, x_sf_host[i], nsf, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(base + h.idx, topk_idx_host[i], nk, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(base + h.w, topk_w_host[i], nk, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in[b], cin);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev_in[b], 0);
+    // slot b's y is overwritten once batch i - 2's copy-out has read it
+    if (e == cudaSuccess && i >= 2) e = cudaStreamWaitEvent(s, ev_out[b], 0);
+    st = cuda_status(e);
+    if (st != MOE_OK) break;
+    const int32_t* idx_d = reinterpret_cast<const int32_t*>(base + h.idx);
+    st = moe_plan(shape, idx_d, workspace, L.total, stream);
+    if (st == MOE_OK)
+      st = moe_forward(shape, base + h.x, reinterpret_cast<const int32_t*>(base + h.x_sf), idx_d,
+                       reinterpret_cast<const float*>(base + h.w), w1_t, w1_sf_t, w2_t, w2_sf_t,
+                       reinterpret_cast<uint16_t*>(base + h.y), workspace, L.total, stream);
+    if (st != MOE_OK) break;
+    e = cudaEventRecord(ev_comp[b], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cout, ev_comp[b], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(y_host[i], base + h.y, ny, cudaMemcpyDeviceToHost, cout);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_out[b], cout);
+    st = cuda_status(e);
+  }
+  // `stream` is ordered after the last copy-out; then drain all three streams
+  // (also after a failure: nothing may still be reading the caller's host
+  // buffers when this returns)
+  if (st == MOE_OK) st = cuda_status(cudaStreamWaitEvent(s, ev_out[(n_batches - 1) & 1], 0));
+  cudaError_t e1 = cin ? cudaStreamSynchronize(cin) : cudaSuccess;
+  cudaError_t e2 = cout ? cudaStreamSynchronize(cout) : cudaSuccess;
+  cudaError_t e3 = cudaStreamSynchronize(s);
+  for (int b = 0; b < 2; ++b) {
+    if (ev_in[b]) cudaEventDestroy(ev_in[b]);
+    if (ev_comp[b]) cudaEventDestroy(ev_comp[b]);
+    if (ev_out[b]) cudaEventDestroy(ev_out[b]);
+  }
+  if (ev_start) cudaEventDestroy(ev_start);
+  if (cin) cudaStreamDestroy(cin);
+  if (cout) cudaStreamDestroy(cout);
+  if (st != MOE_OK) return st;
+  if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 void moe_debug_set_fault(int skip_iteration, unsigned long long wait_limit_ns) {
   g_fault_skip_it.store(skip_iteration >= 0 ? skip_iteration + 1 : 0);
   g_fault_wait_ns.store(wait_limit_ns);

@@ -90,25 +90,55 @@ __global__ void requant_debug_kernel(const float* __restrict__ a, int rows, int 
   }
 }
 
+// Order of the tiles of one list (n_mt m-tiles x NT n-tiles): the m-tiles
+// go in chunks of kMChunk, and within a chunk the m-tile index runs fastest.
+// The CTAs working at one time then cover a few n-tiles of many m-tiles of
+// the same expert: each weight slice is read from DRAM about once per chunk
+// and reused from L2 by the chunk's m-tiles, while the chunk's activation rows
+// (kMChunk x 128 rows) stay in L2 across its n-tiles.  idx -> (m-tile list
+// position, n-tile).
+constexpr int kMChunk = 16;
+__device__ __forceinline__ void chunked_tile(int idx, int n_mt, int NT, int& mpos, int& nt) {
+  const int per_chunk = kMChunk * NT;
+  const int c = idx / per_chunk, rem = idx - c * per_chunk;
+  const int in_chunk = min(kMChunk, n_mt - c * kMChunk);  // the last chunk may be short
+  nt = rem / in_chunk;
+  mpos = c * kMChunk + (rem - nt * in_chunk);
+}
+
 // Tile v of a launch with `total` tiles of which `n_mix` are mixed-in narrow
 // tiles: narrow tiles sit at the positions where floor(v * n_mix / total)
 // steps up, so they are spread evenly over the launch and every CTA (which
 // takes every gridDim-th tile) gets its share.  Returns true for a narrow
 // tile; mt / nt: its m-tile and n-tile.
+// The narrow-tile kernel (kChunked false) keeps the plain order: its m-tiles
+// are single small experts that share no weights, and walking one expert's
+// n-tiles on neighbouring CTAs streams its weights in address order.
+template <bool kChunked>
 __device__ __forceinline__ bool decode_tile(int v, int total, int n_mix, int NT,
                                             const GemmArgs& args, int& mt, int& nt) {
+  int mpos;
   if (n_mix == 0) {
-    mt = args.norm_mtiles[v / NT];
-    nt = v - (v / NT) * NT;
+    if (kChunked) {
+      chunked_tile(v, total / NT, NT, mpos, nt);
+    } else {
+      mpos = v / NT;
+      nt = v - mpos * NT;
+    }
+    mt = args.norm_mtiles[mpos];
     return false;
   }
   const long long before = (long long)v * n_mix / total;          // narrow tiles before v
   const long long upto = ((long long)v + 1) * n_mix / total;      // ... up to and with v
   const bool nar = upto > before;
   const int idx = nar ? (int)before : v - (int)before;
-  const int* list = nar ? args.narrow_mtiles : args.norm_mtiles;
-  mt = list[idx / NT];
-  nt = idx - (idx / NT) * NT;
+  if (nar) {
+    mt = args.narrow_mtiles[idx / NT];
+    nt = idx - (idx / NT) * NT;
+  } else {
+    chunked_tile(idx, (total - n_mix) / NT, NT, mpos, nt);
+    mt = args.norm_mtiles[mpos];
+  }
   return nar;
 }
 
@@ -197,7 +227,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         int mt, nt;
-        const bool nar = decode_tile(tile, num_tiles, n_mix, NT, args, mt, nt);
+        const bool nar = decode_tile<!kNarrow>(tile, num_tiles, n_mix, NT, args, mt, nt);
         const int e = args.tile_expert[mt];
         const int n0 = nt * kBlockN;
         const bool two_chunks = n_rows - n0 > 128;  // 256 weight rows (else the 128-row tail)
@@ -237,7 +267,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++ti) {
         int mt, nt;
-        (void)decode_tile(tile, num_tiles, n_mix, NT, args, mt, nt);
+        (void)decode_tile<!kNarrow>(tile, num_tiles, n_mix, NT, args, mt, nt);
         const int n_tile = min(kBlockN, n_rows - nt * kBlockN);
         const uint32_t idesc0 = idesc_mxf8f6f4(/*A E4M3*/ 0, /*B E2M1*/ 5, kBlockM, n_tile);
         if (!mbar_wait_or_abort(acc_empty, (ti & 1) ^ 1, 2 * lim, abort_flag)) {
@@ -293,7 +323,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int ti = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++ti) {
       int mt, nt;
-      (void)decode_tile(tile, num_tiles, n_mix, NT, args, mt, nt);
+      (void)decode_tile<!kNarrow>(tile, num_tiles, n_mix, NT, args, mt, nt);
       // warp-uniform decision: every lane leaves or every lane continues
       const bool ready =
           __all_sync(0xffffffffu, mbar_wait_or_abort(acc_full, ti & 1, 2 * lim, abort_flag));

@@ -196,6 +196,31 @@ moe_status moe_forward_host(const moe_shape* shape, const uint8_t* x_host,
                             const void* w2_t, const void* w2_sf_t, uint16_t* y_host,
                             void* workspace, size_t ws_bytes, moe_stream_t stream);
 
+/* A sequence of n_batches independent host-buffer forwards of one shape, for
+ * a caller that feeds successive micro-batches from host memory.  Batch i
+ * reads x_host[i], x_sf_host[i], topk_idx_host[i], topk_w_host[i] and writes
+ * y_host[i] (HOST arrays of HOST pointers, layouts as for moe_forward_host;
+ * batches may share input buffers; a y buffer that several batches share
+ * ends up holding the last of them).  The copies run on two streams of
+ * the call's own: batch i + 1's inputs go up and batch i - 1's y comes down
+ * while batch i's kernels run on `stream`, through two staging slots at the
+ * end of `workspace`, which needs moe_workspace_bytes_host_pipelined(shape)
+ * bytes.  The copies only overlap when the host buffers are pinned; pageable
+ * buffers give the same results at the speed of moe_forward_host.  The call
+ * creates two streams and seven events and destroys them before it returns;
+ * it returns after every copy-out has landed (also when it fails part-way,
+ * with the first error).  n_batches < 0 or a NULL pointer: INVALID_ARG
+ * before anything is enqueued; T == 0 or n_batches == 0: MOE_OK, nothing done. */
+size_t moe_workspace_bytes_host_pipelined(const moe_shape* shape);
+moe_status moe_forward_host_pipelined(const moe_shape* shape, int n_batches,
+                                      const uint8_t* const* x_host,
+                                      const int32_t* const* x_sf_host,
+                                      const int32_t* const* topk_idx_host,
+                                      const float* const* topk_w_host, const void* w1_t,
+                                      const void* w1_sf_t, const void* w2_t,
+                                      const void* w2_sf_t, uint16_t* const* y_host,
+                                      void* workspace, size_t ws_bytes, moe_stream_t stream);
+
 /* ---------------------------------------------------- allocation-free call */
 /* The pages describe no counterpart of this entry point.  It is for callers
  * that cannot call cudaMalloc themselves: a serving runtime whose memory

@@ -96,6 +96,36 @@ def test_invalid_arguments_rejected_without_launch(moe):
     assert lib.moe_debug_requant(256, 4, 33, 256, 256, None) == 2
 
 
+def test_pipelined_host_call_sizes_and_validation(moe):
+    """Two staging slots after the regular workspace; every argument error is
+    reported before anything is enqueued (these calls need no GPU)."""
+    s = moe.shape(64, 256, 512, 8, 2)
+    lib = moe.lib()
+    one, two = moe.moe_workspace_bytes_host(s), moe.moe_workspace_bytes_host_pipelined(s)
+    regular = moe.moe_workspace_bytes(s)
+    assert two - one == one - regular > 0
+    assert moe.moe_workspace_bytes_host_pipelined(moe.shape(64, 200, 512, 8, 2)) == 0
+    vpa = ctypes.c_void_p * 2
+    good, null = vpa(256, 256), vpa(256, None)
+    w = [256] * 4
+
+    def call(n, xs=good, ys=good, ws=4096, ws_bytes=two, shp=s):
+        return lib.moe_forward_host_pipelined(ctypes.byref(shp), n, xs, good, good, good, *w,
+                                              ys, ws, ws_bytes, None)
+    assert call(-1) == 1                       # negative batch count
+    assert call(2, ws=None) == 1               # null workspace
+    assert call(2, ws=4096 + 64) == 1          # misaligned workspace
+    assert call(2, ws_bytes=one) == 3          # room for one staging slot only
+    assert call(2, xs=null) == 1               # a null host pointer in a list
+    assert call(2, ys=null) == 1
+    assert lib.moe_forward_host_pipelined(ctypes.byref(s), 2, None, good, good, good, *w, good,
+                                          4096, two, None) == 1
+    assert call(0) == 0                        # no batches: nothing to do
+    assert call(2, shp=moe.shape(0, 256, 512, 8, 2),
+                ws_bytes=moe.moe_workspace_bytes_host_pipelined(moe.shape(0, 256, 512, 8, 2))) == 0
+    assert call(2, shp=moe.shape(64, 256, 500, 8, 2)) == 2
+
+
 def test_zero_tokens_is_a_no_op(moe):
     s = moe.shape(0, 256, 512, 8, 2)
     ws = moe.moe_workspace_bytes(s)

@@ -174,6 +174,40 @@ def test_host_buffer_entry_point_matches_device_entry_point():
     assert np.array_equal(y_host.numpy().view(np.uint16), y_dev)
 
 
+def test_pipelined_host_entry_point_matches_per_batch_results():
+    """Five batches (three distinct inputs, reused so both staging slots are
+    recycled) through the overlapped host-buffer call: each y equals the
+    device entry point's result for its inputs, bit for bit."""
+    import torch
+
+    import block_scaled_fp8_permute_b200 as moe
+    d = synth.make_inputs(synth.workload("tiny"))
+    T = d["x"].shape[0]
+    perm = np.random.default_rng(11).permutation(T)
+    d_b = dict(d)
+    for key in ("x", "x_sf", "topk_idx", "topk_w"):
+        d_b[key] = np.ascontiguousarray(d[key][perm])
+    d_c = dict(d)
+    d_c["topk_idx"] = np.ascontiguousarray(np.roll(d["topk_idx"], 1, axis=1))  # other routing
+    lay = Layer(d).run()
+    expect = [lay.y_bits(), lay.y_bits()[perm], Layer(d_c).run().y_bits()]
+    pins = []
+    for src in (d, d_b, d_c):
+        pins.append({k: torch.from_numpy(np.ascontiguousarray(src[k])).pin_memory()
+                     for k in ("x", "x_sf", "topk_idx", "topk_w")})
+    order = [0, 1, 2, 0, 1]
+    ys = [torch.full(d["x"].shape, -1, dtype=torch.int16).pin_memory() for _ in order]
+    ws = moe.alloc_workspace(lay.shape, "cuda", host_variant="pipelined")
+    assert ws.numel() > moe.moe_workspace_bytes_host(lay.shape)
+    moe.moe_forward_host_pipelined(lay.shape, [pins[b]["x"] for b in order],
+                                   [pins[b]["x_sf"] for b in order],
+                                   [pins[b]["topk_idx"] for b in order],
+                                   [pins[b]["topk_w"] for b in order], *lay.wt, ys, ws)
+    for i, b in enumerate(order):
+        assert np.array_equal(ys[i].numpy().view(np.uint16), expect[b]), f"batch {i}"
+    assert moe.moe_get_device_status(ws) == 0
+
+
 _WEIGHTS = {}
 
 
