@@ -34,12 +34,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer fwd TFLOPS & tokens/s on 1 B200; % of tensor/HBM roofline"
 
-# DRAM traffic (read + write bytes) of one linear1 launch on the mid workload from one ncu
-# capture (summarised, with its command, under profiles/).  Reported only while the kernel
-# sources still hash to the value they had when the counters were taken; otherwise the
-# traffic is unknown (null).
-LINEAR1_TRAFFIC = {"workload": "mid", "bytes": 110.124032e6 + 9.4336e6,
-                   "sources_sha256_16": "9713771996a5720f"}
+# DRAM traffic (read + write bytes) of one linear1 launch on the usage workload (full size)
+# from one ncu capture (summarised, with its command, under profiles/).  Reported only while
+# the kernel sources still hash to the value they had when the counters were taken;
+# otherwise the traffic is unknown (null).
+LINEAR1_TRAFFIC = {"workload": "usage", "bytes": 1241.526016e6 + 152.760576e6,
+                   "sources_sha256_16": "6b76f8d1d804e3d8"}
 LINEAR1_SOURCES = ["moe_gemm.cu", "moe_epilogue.cuh", "moe_device.cuh", "sm100_ptx.cuh",
                    "moe_internal.cuh"]
 

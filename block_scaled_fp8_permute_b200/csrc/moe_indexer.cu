@@ -41,11 +41,13 @@ constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
 constexpr uint32_t kIdxTmemCols = 512;
 constexpr uint32_t kIdxAccStride = 256;  // accumulator buffer b at column 256 b
 constexpr uint32_t kIdxSfCol = 448;      // scale buffers: SFA at +16b (4 cols), SFB at +16b+4 (8)
-// stage ring, then two weight slots (one per accumulator buffer: the group's
-// kN weights, 768 bytes), then barriers
+// stage ring, then a ring of weight slots (the group's kN weights, up to 768
+// bytes each; four deep, so a slot's bulk load is issued while the epilogue
+// is still three tiles behind it), then barriers
 constexpr size_t kIdxSmemStage = (size_t)kIdxStages * (kIdxSmemA + kIdxSmemB + kSfChunk + kIdxSmemSFB);
 constexpr int kIdxWSlot = 1024;
-constexpr size_t kIdxSmemBytes = kIdxSmemStage + 2 * kIdxWSlot + 256;
+constexpr int kIdxWSlots = 4;
+constexpr size_t kIdxSmemBytes = kIdxSmemStage + kIdxWSlots * kIdxWSlot + 256;
 static_assert(kIdxSmemBytes <= 232448, "shared memory per CTA");
 static_assert(kIdxSmemA % 1024 == 0 && kIdxSmemB % 1024 == 0, "swizzled stage alignment");
 
@@ -111,14 +113,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint8_t* sB = sA + kIdxStages * kIdxSmemA;
   uint8_t* sSFA = sB + kIdxStages * kIdxSmemB;
   uint8_t* sSFB = sSFA + kIdxStages * kSfChunk;
-  float* wslot = reinterpret_cast<float*>(smem_raw + kIdxSmemStage);  // [2][kIdxWSlot / 4]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + kIdxSmemStage + 2 * kIdxWSlot);
+  float* wslot = reinterpret_cast<float*>(smem_raw + kIdxSmemStage);  // [kIdxWSlots][kIdxWSlot / 4]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + kIdxSmemStage + kIdxWSlots * kIdxWSlot);
   uint64_t* empty = full + kIdxStages;
   uint64_t* acc_full = empty + kIdxStages;  // [2]
   uint64_t* acc_empty = acc_full + 2;       // [2]
-  uint64_t* w_full = acc_empty + 2;         // [2] weight slot b loaded
-  uint64_t* w_empty = w_full + 2;           // [2] weight slot b read by every epilogue warp
-  uint64_t* drain = w_empty + 2;
+  uint64_t* w_full = acc_empty + 2;         // [kIdxWSlots] weight slot loaded
+  uint64_t* w_empty = w_full + kIdxWSlots;  // [kIdxWSlots] weight slot read by every epilogue warp
+  uint64_t* drain = w_empty + kIdxWSlots;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -131,6 +133,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kIdxEpiWarps);
+    }
+    for (int b = 0; b < kIdxWSlots; ++b) {
       mbar_init(&w_full[b], 1);
       mbar_init(&w_empty[b], kIdxEpiWarps);
     }
@@ -157,121 +161,140 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint32_t issued_mask = 0, last_phase = 0;
   uint32_t w_issued = 0, w_phase = 0;  // weight slots loaded (producer lane), for the failure path
 
+  // This CTA's tiles are blockIdx.x + k * gridDim.x, k = 0 .. n_mine - 1.
+  // Every role walks them in batches of 32: each lane reads the activity flag
+  // of one tile of the next batch while the current batch is worked through,
+  // and a ballot turns the 32 flags into a mask, so no tile waits on a global
+  // load.
+  const long long n_mine =
+      num_tiles > (int)blockIdx.x ? (num_tiles - (long long)blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  auto act_flag = [&](long long k) -> uint32_t {
+    const long long t = blockIdx.x + k * gridDim.x;
+    return (k < n_mine && t < num_tiles) ? (uint32_t)args.act[t] : 0u;
+  };
+  auto tile_of = [&](long long k) -> int { return (int)(blockIdx.x + k * gridDim.x); };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t it = 0;
-      int tp = 0;  // active tiles so far
-      bool ok = true;
-      const uint32_t tx = kIdxTxA + kN * 128 + kSfChunk + kIdxSmemSFB;
-      bool act = blockIdx.x < num_tiles && args.act[blockIdx.x];
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int nt = tile + gridDim.x;
-        const bool nact = nt < num_tiles && args.act[nt];  // loaded while this tile is issued
-        const bool cur = act;
-        act = nact;
-        if (!cur) continue;
-        const int g = tile / args.n_tiles_k, kt = tile - g * args.n_tiles_k;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % kIdxStages;
-          const uint32_t ph = (it / kIdxStages) & 1;
-          if (!mbar_wait_or_abort(&empty[s], ph ^ 1, 2 * kWaitLimitNs, abort_flag)) {
-            if (!*abort_flag) record_timeout(args.hdr, 110);
-            *abort_flag = 1;
-            ok = false;
-            break;
+    uint32_t it = 0;
+    int tp = 0;  // active tiles so far
+    bool ok = true;
+    const uint32_t tx = kIdxTxA + kN * 128 + kSfChunk + kIdxSmemSFB;
+    uint32_t fnext = act_flag(lane);
+    for (long long k0 = 0; k0 < n_mine && ok; k0 += 32) {
+      uint32_t mask = __ballot_sync(0xffffffffu, fnext != 0);
+      fnext = act_flag(k0 + 32 + lane);
+      while (mask != 0 && ok) {
+        const int tile = tile_of(k0 + __ffs(mask) - 1);
+        mask &= mask - 1;
+        if (lane == 0) {
+          const int g = tile / args.n_tiles_k, kt = tile - g * args.n_tiles_k;
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const int s = it % kIdxStages;
+            const uint32_t ph = (it / kIdxStages) & 1;
+            if (!mbar_wait_or_abort(&empty[s], ph ^ 1, 2 * kWaitLimitNs, abort_flag)) {
+              if (!*abort_flag) record_timeout(args.hdr, 110);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[s], tx);
+            tma_load_3d(sA + s * kIdxSmemA, &tmK, &full[s], 0, kt * 128, kb);
+            tma_load_2d(sB + s * kIdxSmemB, &tmQ, &full[s], kb * 128, g * kN);
+            bulk_load(sSFA + s * kSfChunk,
+                      args.sfa + ((size_t)kb * args.n_tiles_k + kt) * kSfChunk, kSfChunk, &full[s]);
+            bulk_load(sSFB + s * kIdxSmemSFB, args.sfb + ((size_t)g * KB + kb) * kIdxSmemSFB,
+                      kIdxSmemSFB, &full[s]);
+            issued_mask |= 1u << s;
+            last_phase = (last_phase & ~(1u << s)) | (ph << s);
           }
-          mbar_arrive_expect_tx(&full[s], tx);
-          tma_load_3d(sA + s * kIdxSmemA, &tmK, &full[s], 0, kt * 128, kb);
-          tma_load_2d(sB + s * kIdxSmemB, &tmQ, &full[s], kb * 128, g * kN);
-          bulk_load(sSFA + s * kSfChunk,
-                    args.sfa + ((size_t)kb * args.n_tiles_k + kt) * kSfChunk, kSfChunk, &full[s]);
-          bulk_load(sSFB + s * kIdxSmemSFB, args.sfb + ((size_t)g * KB + kb) * kIdxSmemSFB,
-                    kIdxSmemSFB, &full[s]);
-          issued_mask |= 1u << s;
-          last_phase = (last_phase & ~(1u << s)) | (ph << s);
+          if (ok) {
+            // the group's weights into the next slot of the weight ring (rows
+            // of tokens past S are not read: the slot keeps stale values there)
+            const int b = tp % kIdxWSlots;
+            const uint32_t wpar = (uint32_t)(tp / kIdxWSlots) & 1u;
+            if (!mbar_wait_or_abort(&w_empty[b], wpar ^ 1, 2 * kWaitLimitNs, abort_flag)) {
+              if (!*abort_flag) record_timeout(args.hdr, 111);
+              *abort_flag = 1;
+              ok = false;
+            } else {
+              const int ntok = min(kTok, args.S - g * kTok);
+              const uint32_t wbytes = (uint32_t)(ntok * kHh * 4);
+              mbar_arrive_expect_tx(&w_full[b], wbytes);
+              bulk_load(wslot + b * (kIdxWSlot / 4), args.w + (size_t)g * kN, wbytes, &w_full[b]);
+              w_issued |= 1u << b;
+              w_phase = (w_phase & ~(1u << b)) | (wpar << b);
+              ++tp;
+            }
+          }
         }
-        if (!ok) break;
-        // the group's weights into the slot of this tile's accumulator buffer
-        // (rows of tokens past S are not read: the slot keeps stale values there)
-        const int b = tp & 1;
-        if (!mbar_wait_or_abort(&w_empty[b], ((tp >> 1) & 1) ^ 1, 2 * kWaitLimitNs, abort_flag)) {
-          if (!*abort_flag) record_timeout(args.hdr, 111);
-          *abort_flag = 1;
-          ok = false;
-          break;
-        }
-        const int ntok = min(kTok, args.S - g * kTok);
-        const uint32_t wbytes = (uint32_t)(ntok * kHh * 4);
-        mbar_arrive_expect_tx(&w_full[b], wbytes);
-        bulk_load(wslot + b * (kIdxWSlot / 4), args.w + (size_t)g * kN, wbytes, &w_full[b]);
-        w_issued |= 1u << b;
-        w_phase = (w_phase & ~(1u << b)) | ((uint32_t)((tp >> 1) & 1) << b);
-        ++tp;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
-      uint32_t it = 0;
-      int ta = 0;  // active tiles so far
-      bool issued_any = false, ok = true;
-      const uint32_t idesc0 = idesc_mxf8f6f4(/*A E2M1*/ 5, /*B E4M3*/ 0, 128, kN);
-      const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA)), b_desc0 = sdesc_sw128(smem_u32(sB));
-      const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
-      bool act = blockIdx.x < num_tiles && args.act[blockIdx.x];
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int nt = tile + gridDim.x;
-        const bool nact = nt < num_tiles && args.act[nt];  // loaded while this tile is issued
-        const bool cur = act;
-        act = nact;
-        if (!cur) continue;
-        const int b = ta & 1;
-        if (!mbar_wait_or_abort(&acc_empty[b], ((ta >> 1) & 1) ^ 1, 2 * kWaitLimitNs,
-                                abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t acc = tmem + kIdxAccStride * (uint32_t)b;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % kIdxStages;
-          const uint32_t ph = (it / kIdxStages) & 1;
-          if (!mbar_wait_or_abort(&full[s], ph, kWaitLimitNs, abort_flag)) {
+    uint32_t it = 0;
+    int ta = 0;  // active tiles so far
+    bool issued_any = false, ok = true;
+    const uint32_t idesc0 = idesc_mxf8f6f4(/*A E2M1*/ 5, /*B E4M3*/ 0, 128, kN);
+    const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA)), b_desc0 = sdesc_sw128(smem_u32(sB));
+    const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
+    uint32_t fnext = act_flag(lane);
+    for (long long k0 = 0; k0 < n_mine && ok; k0 += 32) {
+      uint32_t mask = __ballot_sync(0xffffffffu, fnext != 0);
+      fnext = act_flag(k0 + 32 + lane);
+      // only the count of active tiles matters here: the stages arrive in order
+      for (int n = __popc(mask); n > 0 && ok; --n) {
+        if (lane == 0) {
+          const int b = ta & 1;
+          if (!mbar_wait_or_abort(&acc_empty[b], ((ta >> 1) & 1) ^ 1, 2 * kWaitLimitNs,
+                                  abort_flag)) {
             ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sfa_t = tmem + kIdxSfCol + 16u * (it & 1u);
-          const uint32_t sfb_t = sfa_t + 4u;
-          tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + (uint64_t)((s * kSfChunk) >> 4));
-          tc_cp_32x128b_warpx4(sfb_t, sfb_desc0 + (uint64_t)((s * kIdxSmemSFB) >> 4));
-          if (kN > 128)
-            tc_cp_32x128b_warpx4(sfb_t + 4u,
-                                 sfb_desc0 + (uint64_t)((s * kIdxSmemSFB + kSfChunk) >> 4));
-          const uint64_t adesc = a_desc0 + (uint64_t)((s * kIdxSmemA) >> 4);
-          const uint64_t bdesc = b_desc0 + (uint64_t)((s * kIdxSmemB) >> 4);
+          } else {
+            tc_fence_after();
+            const uint32_t acc = tmem + kIdxAccStride * (uint32_t)b;
+            for (int kb = 0; kb < KB; ++kb, ++it) {
+              const int s = it % kIdxStages;
+              const uint32_t ph = (it / kIdxStages) & 1;
+              if (!mbar_wait_or_abort(&full[s], ph, kWaitLimitNs, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t sfa_t = tmem + kIdxSfCol + 16u * (it & 1u);
+              const uint32_t sfb_t = sfa_t + 4u;
+              tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + (uint64_t)((s * kSfChunk) >> 4));
+              tc_cp_32x128b_warpx4(sfb_t, sfb_desc0 + (uint64_t)((s * kIdxSmemSFB) >> 4));
+              if (kN > 128)
+                tc_cp_32x128b_warpx4(sfb_t + 4u,
+                                     sfb_desc0 + (uint64_t)((s * kIdxSmemSFB + kSfChunk) >> 4));
+              const uint64_t adesc = a_desc0 + (uint64_t)((s * kIdxSmemA) >> 4);
+              const uint64_t bdesc = b_desc0 + (uint64_t)((s * kIdxSmemB) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t id = idesc_with_sf_id(idesc0, kk, kk);
-            mma_mxf8f6f4(acc, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id,
-                         (kb | kk) != 0 ? 1u : 0u, sfa_t | ((uint32_t)kk << 30),
-                         sfb_t | ((uint32_t)kk << 30));
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t id = idesc_with_sf_id(idesc0, kk, kk);
+                mma_mxf8f6f4(acc, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id,
+                             (kb | kk) != 0 ? 1u : 0u, sfa_t | ((uint32_t)kk << 30),
+                             sfb_t | ((uint32_t)kk << 30));
+              }
+              issued_any = true;
+              tc_commit(&empty[s]);
+            }
+            if (ok) {
+              tc_commit(&acc_full[b]);
+              ++ta;
+            }
           }
-          issued_any = true;
-          tc_commit(&empty[s]);
         }
-        if (!ok) break;
-        tc_commit(&acc_full[b]);
-        ++ta;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
-      if (!ok) {
-        if (!*abort_flag) record_timeout(args.hdr, 120);
-        *abort_flag = 1;
-        if (issued_any) {  // wait for the MMAs in flight before TMEM is released
-          tc_commit(drain);
-          (void)mbar_wait(drain, 0);
-        }
+    }
+    if (lane == 0 && !ok) {
+      if (!*abort_flag) record_timeout(args.hdr, 120);
+      *abort_flag = 1;
+      if (issued_any) {  // wait for the MMAs in flight before TMEM is released
+        tc_commit(drain);
+        (void)mbar_wait(drain, 0);
       }
     }
   } else {
@@ -283,96 +306,111 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     constexpr int kMine = (kTok + 2) / 3;
     int ta = 0;
-    bool act_next = blockIdx.x < num_tiles && args.act[blockIdx.x];
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int g = tile / args.n_tiles_k, kt = tile - g * args.n_tiles_k;
-      const int j = kt * 128 + r;
-      const bool active = act_next;
-      act_next = tile + (int)gridDim.x < num_tiles && args.act[tile + gridDim.x];
-      // key ranges of this warp's tokens (loaded before the waits)
-      int lo[kMine], hi[kMine];
+    bool dead = false;
+    uint32_t fnext = act_flag(lane);
+    for (long long k0 = 0; k0 < n_mine && !dead; k0 += 32) {
+      const uint32_t mask = __ballot_sync(0xffffffffu, fnext != 0);
+      fnext = act_flag(k0 + 32 + lane);
+      const int nb = (int)(n_mine - k0 < 32 ? n_mine - k0 : 32);
+      for (int bit = 0; bit < nb; ++bit) {
+        const int tile = tile_of(k0 + bit);
+        const int g = tile / args.n_tiles_k, kt = tile - g * args.n_tiles_k;
+        const int j = kt * 128 + r;
+        const bool active = (mask >> bit) & 1u;
+        // key ranges of this warp's tokens (loaded before the waits)
+        int lo[kMine], hi[kMine];
 #pragma unroll
-      for (int m = 0; m < kMine; ++m) {
-        const int i = g * kTok + h + 3 * m;
-        const bool tok = h + 3 * m < kTok && i < args.S;
-        lo[m] = tok ? max(__ldg(args.ks + i), 0) : 0;
-        hi[m] = tok ? min(__ldg(args.ke + i), args.N) : 0;
-      }
-      const int b = ta & 1;
-      bool use = false;  // this tile's accumulator (and weight slot) is read
-      if (active) {
-        const uint32_t par = (ta >> 1) & 1;
-        const bool ready = __all_sync(0xffffffffu,
-                                      mbar_wait_or_abort(&acc_full[b], par, 2 * kWaitLimitNs, abort_flag) &&
-                                          mbar_wait_or_abort(&w_full[b], par, 2 * kWaitLimitNs, abort_flag));
-        if (!ready) {
-          if (lane == 0) {
-            if (!*abort_flag) record_timeout(args.hdr, 130);
-            *abort_flag = 1;
-          }
-          break;
+        for (int m = 0; m < kMine; ++m) {
+          const int i = g * kTok + h + 3 * m;
+          const bool tok = active && h + 3 * m < kTok && i < args.S;
+          lo[m] = tok ? max(__ldg(args.ks + i), 0) : 0;
+          hi[m] = tok ? min(__ldg(args.ke + i), args.N) : 0;
         }
-        tc_fence_after();
-        use = true;
-      }
-      const float* w_s = wslot + b * (kIdxWSlot / 4);
-      // this warp's tokens t = h + 3m, in column chunks of at most 64: every
-      // TMEM load of a chunk first, one wait, then the weighted ReLU sums on
-      // eight independent accumulator chains
-      constexpr int kC = kHh > 64 ? 64 : kHh;  // columns per chunk
-      float acc[kMine][8];
+        const int b = ta & 1;            // accumulator buffer
+        const int wb = ta % kIdxWSlots;  // weight slot
+        bool use = false;  // this tile's accumulator (and weight slot) is read
+        if (active) {
+          const uint32_t par = (ta >> 1) & 1, wpar = (uint32_t)(ta / kIdxWSlots) & 1u;
+          const bool ready =
+              __all_sync(0xffffffffu,
+                         mbar_wait_or_abort(&acc_full[b], par, 2 * kWaitLimitNs, abort_flag) &&
+                             mbar_wait_or_abort(&w_full[wb], wpar, 2 * kWaitLimitNs, abort_flag));
+          if (!ready) {
+            if (lane == 0) {
+              if (!*abort_flag) record_timeout(args.hdr, 130);
+              *abort_flag = 1;
+            }
+            dead = true;
+            break;
+          }
+          tc_fence_after();
+          use = true;
+        }
+        const float* w_s = wslot + wb * (kIdxWSlot / 4);
+        // this warp's tokens t = h + 3m, in column chunks of at most 64: every
+        // TMEM load of a chunk first, one wait, then the weighted ReLU sums on
+        // eight independent accumulator chains (head c goes to chain c % 8),
+        // two chains per packed FP32x2 instruction
+        constexpr int kC = kHh > 64 ? 64 : kHh;  // columns per chunk
+        uint64_t acc[kMine][4];
 #pragma unroll
-      for (int m = 0; m < kMine; ++m)
+        for (int m = 0; m < kMine; ++m)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) acc[m][u] = 0.0f;
+          for (int u = 0; u < 4; ++u) acc[m][u] = 0ull;
 #pragma unroll
-      for (int c0 = 0; c0 < kHh; c0 += kC) {
-        uint32_t v[kMine][kC];
-        if (use) {  // warp-uniform: the TMEM loads are collective
+        for (int c0 = 0; c0 < kHh; c0 += kC) {
+          uint32_t v[kMine][kC];
+          if (use) {  // warp-uniform: the TMEM loads are collective
 #pragma unroll
-          for (int m = 0; m < kMine; ++m)
-            if (h + 3 * m < kTok)
-              load_head_cols<kC>(trow + kIdxAccStride * (uint32_t)b +
-                                     (uint32_t)((h + 3 * m) * kHh + c0), v[m]);
-          tc_wait_ld();
+            for (int m = 0; m < kMine; ++m)
+              if (h + 3 * m < kTok)
+                load_head_cols<kC>(trow + kIdxAccStride * (uint32_t)b +
+                                       (uint32_t)((h + 3 * m) * kHh + c0), v[m]);
+            tc_wait_ld();
 #pragma unroll
-          for (int m = 0; m < kMine; ++m) {
-            const int t = h + 3 * m;
-            if (t < kTok) {
-              const float4* wt = reinterpret_cast<const float4*>(w_s + t * kHh + c0);
+            for (int m = 0; m < kMine; ++m) {
+              const int t = h + 3 * m;
+              if (t < kTok) {
+                const ulonglong2* wt = reinterpret_cast<const ulonglong2*>(w_s + t * kHh + c0);
 #pragma unroll
-              for (int h4 = 0; h4 < kC / 4; ++h4) {
-                const float4 w4 = wt[h4];
-                const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  acc[m][(4 * h4 + u) & 7] = fmaf(wv[u], fmaxf(__uint_as_float(v[m][4 * h4 + u]), 0.0f),
-                                                  acc[m][(4 * h4 + u) & 7]);
+                for (int h4 = 0; h4 < kC / 4; ++h4) {
+                  const ulonglong2 w4 = wt[h4];  // heads c0 + 4 h4 .. + 3, two per word
+                  const uint64_t x01 = relu_pack_f32x2(v[m][4 * h4], v[m][4 * h4 + 1]);
+                  const uint64_t x23 = relu_pack_f32x2(v[m][4 * h4 + 2], v[m][4 * h4 + 3]);
+                  acc[m][(2 * h4) & 3] = fma_f32x2(w4.x, x01, acc[m][(2 * h4) & 3]);
+                  acc[m][(2 * h4 + 1) & 3] = fma_f32x2(w4.y, x23, acc[m][(2 * h4 + 1) & 3]);
+                }
               }
             }
           }
         }
-      }
-      if (use) {  // accumulator and weights are in registers: release both
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&acc_empty[b]);
-          mbar_arrive(&w_empty[b]);
+        if (use) {  // accumulator and weights are in registers: release both
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&acc_empty[b]);
+            mbar_arrive(&w_empty[wb]);
+          }
         }
-      }
 #pragma unroll
-      for (int m = 0; m < kMine; ++m) {
-        const int t = h + 3 * m;
-        const int i = g * kTok + t;
-        const bool here = t < kTok && i < args.S && j < args.N;  // an entry of the output
-        const bool scored = use && here && j >= lo[m] && j < hi[m];
-        const float logit = scored ? ((acc[m][0] + acc[m][1]) + (acc[m][2] + acc[m][3])) +
-                                         ((acc[m][4] + acc[m][5]) + (acc[m][6] + acc[m][7]))
-                                   : -INFINITY;
-        if (scored || (here && args.clean)) args.out[(size_t)i * args.N + j] = logit;
+        for (int m = 0; m < kMine; ++m) {
+          const int t = h + 3 * m;
+          const int i = g * kTok + t;
+          const bool here = t < kTok && i < args.S && j < args.N;  // an entry of the output
+          const bool scored = use && here && j >= lo[m] && j < hi[m];
+          float a8[8];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            a8[2 * u] = __uint_as_float((uint32_t)acc[m][u]);
+            a8[2 * u + 1] = __uint_as_float((uint32_t)(acc[m][u] >> 32));
+          }
+          const float logit = scored ? ((a8[0] + a8[1]) + (a8[2] + a8[3])) +
+                                           ((a8[4] + a8[5]) + (a8[6] + a8[7]))
+                                     : -INFINITY;
+          if (scored || (here && args.clean)) args.out[(size_t)i * args.N + j] = logit;
+        }
+        if (active) ++ta;
       }
-      if (active) ++ta;
     }
   }
 
@@ -383,7 +421,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // copies issued that nobody consumed land before the CTA's memory goes away
     for (int s = 0; s < kIdxStages; ++s)
       if (issued_mask & (1u << s)) (void)mbar_wait(&full[s], (last_phase >> s) & 1);
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < kIdxWSlots; ++b)
       if (w_issued & (1u << b)) (void)mbar_wait(&w_full[b], (w_phase >> b) & 1);
   }
   if (warp == 1) {

@@ -209,6 +209,19 @@ __device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sd
                : "memory");
 }
 
+// Two FP32 lanes packed in 64 bits (lane 0 in the low word): d = a * b + c
+// rounded to nearest per lane, one instruction for both.
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// max(x, 0) of two FP32 bit patterns, packed as above
+__device__ __forceinline__ uint64_t relu_pack_f32x2(uint32_t lo, uint32_t hi) {
+  const float a = fmaxf(__uint_as_float(lo), 0.0f), b = fmaxf(__uint_as_float(hi), 0.0f);
+  return (uint64_t)__float_as_uint(a) | ((uint64_t)__float_as_uint(b) << 32);
+}
+
 __device__ __forceinline__ void tc_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
