@@ -15,9 +15,20 @@
 // is a per-thread loop, no cross-lane reduction.  That sum costs about as
 // much as the tile's MMAs, so the accumulator is double-buffered in TMEM
 // (two 192-column buffers) and the MMAs of one tile run while the epilogue
-// reduces the previous one.  One CTA per SM, persistent, 320 threads:
-//   warp 0     TMA producer: key tile 128 x 128 (E2M1, unpacked by the TMA),
-//              query tile kN x 128 (E4M3), their scale chunks; 4-stage ring
+// reduces the previous one.
+//
+// Work order.  A unit is a run of up to C consecutive key tiles of one query
+// group; units are numbered chunk-major (unit = chunk * n_groups + group), and
+// CTA c takes units c, c + grid, ...  A CTA therefore meets the same query
+// group for up to C tiles in a row, and the group's query block (kN rows x D,
+// with its scales) is loaded once into a query slot and read by all of them;
+// only the 8 KB key tile streams per tile.  Without that, the query block was
+// most of the bytes a tile moved into shared memory, and the kernel was bound
+// by those loads.  One CTA per SM, persistent, 448 threads:
+//   warp 0     TMA producer: query blocks into 1-2 query slots (one per group
+//              change), key tiles 128 x 128 (E2M1, unpacked by the TMA) with
+//              their scale chunk into a ring of up to 8 stages, and the
+//              group's head weights into a 4-deep weight ring
 //   warp 1     TMEM allocator and MMA issuer (tcgen05.mma kind::mxf8f6f4,
 //              A = keys E2M1, B = queries E4M3, M=128, N=kN, K=32)
 //   warps 2-13 epilogue: three warps per 32-lane TMEM subpartition, the
@@ -31,28 +42,56 @@
 namespace moe {
 namespace {
 
-constexpr int kIdxStages = 4;
+constexpr int kIdxMaxStages = 8;
 constexpr int kIdxSmemA = 128 * 128;   // keys, one byte per E2M1 element
-constexpr int kIdxSmemB = 192 * 128;   // queries (up to 192 rows), E4M3
-constexpr int kIdxSmemSFB = 2 * kSfChunk;
+constexpr int kIdxQBlock = 192 * 128;  // one K-block of a query block (up to 192 rows), E4M3
+constexpr int kIdxSfbBlock = 2 * kSfChunk;  // the query scales of one K-block
 constexpr int kIdxTxA = 128 * 128 / 2; // bytes the TMA moves for the packed keys
 constexpr int kIdxEpiWarps = 12;  // three per 32-lane TMEM subpartition
 constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
 constexpr uint32_t kIdxTmemCols = 512;
 constexpr uint32_t kIdxAccStride = 256;  // accumulator buffer b at column 256 b
-constexpr uint32_t kIdxSfCol = 448;      // scale buffers: SFA at +16b (4 cols), SFB at +16b+4 (8)
-// stage ring, then a ring of weight slots (the group's kN weights, up to 768
-// bytes each; four deep, so a slot's bulk load is issued while the epilogue
-// is still three tiles behind it), then barriers
-constexpr size_t kIdxSmemStage = (size_t)kIdxStages * (kIdxSmemA + kIdxSmemB + kSfChunk + kIdxSmemSFB);
-constexpr int kIdxWSlot = 1024;
+constexpr uint32_t kIdxSfCol = 448;      // scale buffers: SFA at +16x (4 cols), SFB at +16x+4 (8)
+constexpr int kIdxWSlot = 1024;          // the group's kN weights, up to 768 bytes
 constexpr int kIdxWSlots = 4;
-constexpr size_t kIdxSmemBytes = kIdxSmemStage + kIdxWSlots * kIdxWSlot + 256;
-static_assert(kIdxSmemBytes <= 232448, "shared memory per CTA");
-static_assert(kIdxSmemA % 1024 == 0 && kIdxSmemB % 1024 == 0, "swizzled stage alignment");
+constexpr int kIdxSmemMax = 232448;      // shared memory per CTA
+constexpr int kIdxBarBytes = 512;
+// stage info words (producer -> MMA thread)
+constexpr int kStFirst = 1;   // the tile's first K-block: take the next accumulator buffer
+constexpr int kStLast = 2;    // the tile's last K-block: hand the accumulator to the epilogue
+constexpr int kStNewQ = 4;    // the tile starts a new query group: take the next query slot
+constexpr int kStEnd = 8;     // no more work (a stage without loads)
+constexpr int kStRelQ = 16;   // release the current query slot (a stage without loads)
+static_assert(kIdxSmemA % 1024 == 0 && kIdxQBlock % 1024 == 0, "swizzled block alignment");
 
 // tokens per tile for Hh heads: kN = kTok * Hh query rows on the MMA's N side
 __host__ __device__ constexpr int idx_tokens(int Hh) { return Hh >= 128 ? 1 : 192 / Hh; }
+
+// Shared-memory plan for KB K-blocks: key stages (16 KB of unpacked codes +
+// one 512-byte scale chunk each) and query slots (KB blocks of 24 KB + KB
+// scale pairs of 1 KB).  Two query slots when they leave room for two key
+// stages, else one; then as many key stages as fit, at most 8.
+struct IdxSmem {
+  int stages, qslots;
+  int a_off, q_off, sfa_off, sfb_off, w_off, bar_off, total;
+};
+__host__ __device__ inline IdxSmem idx_smem(int KB) {
+  IdxSmem p{};
+  const int stage = kIdxSmemA + kSfChunk;
+  const int qslot = KB * (kIdxQBlock + kIdxSfbBlock);
+  const int avail = kIdxSmemMax - kIdxWSlots * kIdxWSlot - kIdxBarBytes;
+  p.qslots = (2 * qslot + 2 * stage <= avail) ? 2 : 1;
+  p.stages = (avail - p.qslots * qslot) / stage;
+  if (p.stages > kIdxMaxStages) p.stages = kIdxMaxStages;
+  p.a_off = 0;
+  p.q_off = p.a_off + p.stages * kIdxSmemA;
+  p.sfa_off = p.q_off + p.qslots * KB * kIdxQBlock;
+  p.sfb_off = p.sfa_off + p.stages * kSfChunk;
+  p.w_off = p.sfb_off + p.qslots * KB * kIdxSfbBlock;
+  p.bar_off = p.w_off + kIdxWSlots * kIdxWSlot;
+  p.total = p.bar_off + kIdxBarBytes;
+  return p;
+}
 
 struct IdxArgs {
   const uint8_t* sfa;    // key scale chunks [KB][ceil(N/128)][512]
@@ -66,6 +105,9 @@ struct IdxArgs {
   int S, Hh, N, KB, clean;
   int n_tiles_k;         // ceil(N / 128)
   int n_groups;          // ceil(S / tokens per tile)
+  int chunk_log2;        // C = 2^chunk_log2 key tiles per unit (1..16)
+  int n_chunks;          // ceil(n_tiles_k / C)
+  int n_units;           // n_groups * n_chunks (< 2^28 for the supported shapes)
 };
 
 // Does any token of query group g see a key of key tile kt?  (Decided the
@@ -96,6 +138,26 @@ __device__ __forceinline__ void load_head_cols(uint32_t taddr, uint32_t (&v)[kHh
   }
 }
 
+// Unit m of this CTA (u = blockIdx.x + m * gridDim.x): its group g = u %
+// n_groups and first key tile kt0 = (u / n_groups) * C.  False past the last
+// unit.  (32-bit: u < n_units + gridDim.x.)
+__device__ __forceinline__ bool cta_unit(const IdxArgs& a, int m, int& g, int& kt0) {
+  const int u = (int)blockIdx.x + m * (int)gridDim.x;
+  if (u >= a.n_units) return false;
+  const int c = u / a.n_groups;
+  g = u - c * a.n_groups;
+  kt0 = c << a.chunk_log2;
+  return true;
+}
+// The k-th tile of this CTA: tile k % C of unit k / C.  False when it lies
+// past the last unit or past the last key tile.
+__device__ __forceinline__ bool cta_tile(const IdxArgs& a, long long k, int& g, int& kt) {
+  int kt0;
+  if (!cta_unit(a, (int)(k >> a.chunk_log2), g, kt0)) return false;
+  kt = kt0 + (int)(k & ((1 << a.chunk_log2) - 1));
+  return kt < a.n_tiles_k;
+}
+
 template <int kHh>  // heads per query token (16, 32, 64 or 128)
 __global__ void __launch_bounds__(kIdxThreads, 1)
     mqa_logits_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -109,28 +171,38 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     if (threadIdx.x == 0) set_status(args.hdr, MOE_ERR_CUDA);
     return;
   }
-  uint8_t* sA = smem_raw;
-  uint8_t* sB = sA + kIdxStages * kIdxSmemA;
-  uint8_t* sSFA = sB + kIdxStages * kIdxSmemB;
-  uint8_t* sSFB = sSFA + kIdxStages * kSfChunk;
-  float* wslot = reinterpret_cast<float*>(smem_raw + kIdxSmemStage);  // [kIdxWSlots][kIdxWSlot / 4]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + kIdxSmemStage + kIdxWSlots * kIdxWSlot);
-  uint64_t* empty = full + kIdxStages;
-  uint64_t* acc_full = empty + kIdxStages;  // [2]
-  uint64_t* acc_empty = acc_full + 2;       // [2]
-  uint64_t* w_full = acc_empty + 2;         // [kIdxWSlots] weight slot loaded
-  uint64_t* w_empty = w_full + kIdxWSlots;  // [kIdxWSlots] weight slot read by every epilogue warp
+  const int KB = args.KB;
+  const IdxSmem L = idx_smem(KB);
+  const int NS = L.stages, NQ = L.qslots;
+  uint8_t* sA = smem_raw + L.a_off;      // [NS][128 x 128]
+  uint8_t* sQ = smem_raw + L.q_off;      // [NQ][KB][kN x 128]
+  uint8_t* sSFA = smem_raw + L.sfa_off;  // [NS][512]
+  uint8_t* sSFB = smem_raw + L.sfb_off;  // [NQ][KB][1 KB]
+  float* wslot = reinterpret_cast<float*>(smem_raw + L.w_off);  // [kIdxWSlots][kIdxWSlot / 4]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + L.bar_off);  // [kIdxMaxStages]
+  uint64_t* empty = full + kIdxMaxStages;     // [kIdxMaxStages]
+  uint64_t* q_full = empty + kIdxMaxStages;   // [2] query slot loaded
+  uint64_t* q_empty = q_full + 2;             // [2] query slot no longer read by MMAs
+  uint64_t* acc_full = q_empty + 2;           // [2]
+  uint64_t* acc_empty = acc_full + 2;         // [2]
+  uint64_t* w_full = acc_empty + 2;           // [kIdxWSlots] weight slot loaded
+  uint64_t* w_empty = w_full + kIdxWSlots;    // [kIdxWSlots] weight slot read by every epilogue warp
   uint64_t* drain = w_empty + kIdxWSlots;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  // what the MMA thread does with key stage s (written by the producer before
+  // the stage's loads are issued; read after the stage's full barrier)
+  int* sinfo = const_cast<int*>(abort_flag) + 1;  // [kIdxMaxStages]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kIdxStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kIdxEpiWarps);
     }
@@ -156,145 +228,247 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   const uint32_t tmem = *tmem_holder;
 
   pdl_wait();  // the transformed keys and the query scale chunks come from the previous kernels
-  const int KB = args.KB;
-  const int num_tiles = args.n_tiles_k * args.n_groups;
-  uint32_t issued_mask = 0, last_phase = 0;
-  uint32_t w_issued = 0, w_phase = 0;  // weight slots loaded (producer lane), for the failure path
+  uint32_t issued_mask = 0, last_phase = 0;  // key stages loaded (producer lane), for the failure path
+  uint32_t w_issued = 0, w_phase = 0;        // weight slots loaded
+  uint32_t q_issued = 0, q_phase = 0;        // query slots loaded
 
-  // This CTA's tiles are blockIdx.x + k * gridDim.x, k = 0 .. n_mine - 1.
-  // Every role walks them in batches of 32: each lane reads the activity flag
-  // of one tile of the next batch while the current batch is worked through,
-  // and a ballot turns the 32 flags into a mask, so no tile waits on a global
-  // load.
+  // This CTA's tiles k = 0 .. n_mine - 1 (cta_tile).  Every role walks them
+  // in batches of 32: each lane reads the activity flag of one tile of the
+  // next batch while the current batch is worked through, and a ballot turns
+  // the 32 flags into a mask, so no tile waits on a global load.
   const long long n_mine =
-      num_tiles > (int)blockIdx.x ? (num_tiles - (long long)blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+      args.n_units > (int)blockIdx.x
+          ? (long long)((args.n_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x)
+                << args.chunk_log2
+          : 0;
   auto act_flag = [&](long long k) -> uint32_t {
-    const long long t = blockIdx.x + k * gridDim.x;
-    return (k < n_mine && t < num_tiles) ? (uint32_t)args.act[t] : 0u;
+    int g, kt;
+    if (k >= n_mine || !cta_tile(args, k, g, kt)) return 0u;
+    return (uint32_t)args.act[(size_t)g * args.n_tiles_k + kt];
   };
-  auto tile_of = [&](long long k) -> int { return (int)(blockIdx.x + k * gridDim.x); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    uint32_t it = 0;
-    int tp = 0;  // active tiles so far
+    // Ring positions advance by increments (no division on the per-tile
+    // path); the unit is looked up once per unit.
+    int s = 0, wb = 0, qs = 0;
+    uint32_t ph = 0, w_ph = 0, q_ph = 0;
+    int qe = -1, cur_g = -1, cur_m = -1, g = 0, kt0 = 0;
     bool ok = true;
-    const uint32_t tx = kIdxTxA + kN * 128 + kSfChunk + kIdxSmemSFB;
+    const uint32_t tx = kIdxTxA + kSfChunk;
+    const uint32_t qtx = (uint32_t)KB * (kN * 128 + kIdxSfbBlock);
     uint32_t fnext = act_flag(lane);
     for (long long k0 = 0; k0 < n_mine && ok; k0 += 32) {
       uint32_t mask = __ballot_sync(0xffffffffu, fnext != 0);
       fnext = act_flag(k0 + 32 + lane);
       while (mask != 0 && ok) {
-        const int tile = tile_of(k0 + __ffs(mask) - 1);
+        const long long k = k0 + __ffs(mask) - 1;
         mask &= mask - 1;
         if (lane == 0) {
-          const int g = tile / args.n_tiles_k, kt = tile - g * args.n_tiles_k;
-          for (int kb = 0; kb < KB; ++kb, ++it) {
-            const int s = it % kIdxStages;
-            const uint32_t ph = (it / kIdxStages) & 1;
-            if (!mbar_wait_or_abort(&empty[s], ph ^ 1, 2 * kWaitLimitNs, abort_flag)) {
+          const int m = (int)(k >> args.chunk_log2);
+          if (m != cur_m) {
+            cur_m = m;
+            (void)cta_unit(args, m, g, kt0);  // an active tile: its unit exists
+          }
+          const int kt = kt0 + (int)(k & ((1 << args.chunk_log2) - 1));
+          const bool new_epoch = g != cur_g;
+          if (new_epoch && qe >= 0) {
+            // An info-only stage tells the MMA thread that the current query
+            // slot is read by no later MMA: it releases the slot once the MMAs
+            // issued so far complete.  (With one slot the wait below needs
+            // exactly that release.)
+            if (!mbar_wait_or_abort(&empty[s], ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+              if (!*abort_flag) record_timeout(args.hdr, 114);
+              *abort_flag = 1;
+              ok = false;
+            } else {
+              sinfo[s] = kStRelQ;
+              mbar_arrive(&full[s]);
+              if (++s == NS) {
+                s = 0;
+                ph ^= 1u;
+              }
+              if (++qs == NQ) {
+                qs = 0;
+                q_ph ^= 1u;
+              }
+            }
+          }
+          if (new_epoch && ok) {
+            // a new query group: its query block and scales into the next slot
+            ++qe;
+            cur_g = g;
+            if (!mbar_wait_or_abort(&q_empty[qs], q_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+              if (!*abort_flag) record_timeout(args.hdr, 112);
+              *abort_flag = 1;
+              ok = false;
+            } else {
+              mbar_arrive_expect_tx(&q_full[qs], qtx);
+              for (int kb = 0; kb < KB; ++kb)
+                tma_load_2d(sQ + (size_t)(qs * KB + kb) * kIdxQBlock, &tmQ, &q_full[qs], kb * 128,
+                            g * kN);
+              bulk_load(sSFB + (size_t)qs * KB * kIdxSfbBlock,
+                        args.sfb + (size_t)g * KB * kIdxSfbBlock, (uint32_t)KB * kIdxSfbBlock,
+                        &q_full[qs]);
+              q_issued |= 1u << qs;
+              q_phase = (q_phase & ~(1u << qs)) | (q_ph << qs);
+            }
+          }
+          for (int kb = 0; kb < KB && ok; ++kb) {
+            if (!mbar_wait_or_abort(&empty[s], ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
               if (!*abort_flag) record_timeout(args.hdr, 110);
               *abort_flag = 1;
               ok = false;
               break;
             }
+            sinfo[s] = (kb == 0 ? kStFirst : 0) | (kb == KB - 1 ? kStLast : 0) |
+                       (kb == 0 && new_epoch ? kStNewQ : 0);
             mbar_arrive_expect_tx(&full[s], tx);
-            tma_load_3d(sA + s * kIdxSmemA, &tmK, &full[s], 0, kt * 128, kb);
-            tma_load_2d(sB + s * kIdxSmemB, &tmQ, &full[s], kb * 128, g * kN);
+            tma_load_3d(sA + (size_t)s * kIdxSmemA, &tmK, &full[s], 0, kt * 128, kb);
             bulk_load(sSFA + s * kSfChunk,
                       args.sfa + ((size_t)kb * args.n_tiles_k + kt) * kSfChunk, kSfChunk, &full[s]);
-            bulk_load(sSFB + s * kIdxSmemSFB, args.sfb + ((size_t)g * KB + kb) * kIdxSmemSFB,
-                      kIdxSmemSFB, &full[s]);
             issued_mask |= 1u << s;
             last_phase = (last_phase & ~(1u << s)) | (ph << s);
+            if (++s == NS) {
+              s = 0;
+              ph ^= 1u;
+            }
           }
           if (ok) {
             // the group's weights into the next slot of the weight ring (rows
             // of tokens past S are not read: the slot keeps stale values there)
-            const int b = tp % kIdxWSlots;
-            const uint32_t wpar = (uint32_t)(tp / kIdxWSlots) & 1u;
-            if (!mbar_wait_or_abort(&w_empty[b], wpar ^ 1, 2 * kWaitLimitNs, abort_flag)) {
+            if (!mbar_wait_or_abort(&w_empty[wb], w_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
               if (!*abort_flag) record_timeout(args.hdr, 111);
               *abort_flag = 1;
               ok = false;
             } else {
               const int ntok = min(kTok, args.S - g * kTok);
               const uint32_t wbytes = (uint32_t)(ntok * kHh * 4);
-              mbar_arrive_expect_tx(&w_full[b], wbytes);
-              bulk_load(wslot + b * (kIdxWSlot / 4), args.w + (size_t)g * kN, wbytes, &w_full[b]);
-              w_issued |= 1u << b;
-              w_phase = (w_phase & ~(1u << b)) | (wpar << b);
-              ++tp;
+              mbar_arrive_expect_tx(&w_full[wb], wbytes);
+              bulk_load(wslot + wb * (kIdxWSlot / 4), args.w + (size_t)g * kN, wbytes, &w_full[wb]);
+              w_issued |= 1u << wb;
+              w_phase = (w_phase & ~(1u << wb)) | (w_ph << wb);
+              if (++wb == kIdxWSlots) {
+                wb = 0;
+                w_ph ^= 1u;
+              }
             }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
+    }
+    // one more stage, without loads, tells the MMA thread that the work ends
+    if (lane == 0 && ok) {
+      if (!mbar_wait_or_abort(&empty[s], ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+        if (!*abort_flag) record_timeout(args.hdr, 113);
+        *abort_flag = 1;
+      } else {
+        sinfo[s] = kStEnd;
+        mbar_arrive(&full[s]);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    uint32_t it = 0;
-    int ta = 0;  // active tiles so far
-    bool issued_any = false, ok = true;
-    const uint32_t idesc0 = idesc_mxf8f6f4(/*A E2M1*/ 5, /*B E4M3*/ 0, 128, kN);
-    const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA)), b_desc0 = sdesc_sw128(smem_u32(sB));
-    const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
-    uint32_t fnext = act_flag(lane);
-    for (long long k0 = 0; k0 < n_mine && ok; k0 += 32) {
-      uint32_t mask = __ballot_sync(0xffffffffu, fnext != 0);
-      fnext = act_flag(k0 + 32 + lane);
-      // only the count of active tiles matters here: the stages arrive in order
-      for (int n = __popc(mask); n > 0 && ok; --n) {
-        if (lane == 0) {
-          const int b = ta & 1;
-          if (!mbar_wait_or_abort(&acc_empty[b], ((ta >> 1) & 1) ^ 1, 2 * kWaitLimitNs,
-                                  abort_flag)) {
-            ok = false;
-          } else {
-            tc_fence_after();
-            const uint32_t acc = tmem + kIdxAccStride * (uint32_t)b;
-            for (int kb = 0; kb < KB; ++kb, ++it) {
-              const int s = it % kIdxStages;
-              const uint32_t ph = (it / kIdxStages) & 1;
-              if (!mbar_wait_or_abort(&full[s], ph, kWaitLimitNs, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t sfa_t = tmem + kIdxSfCol + 16u * (it & 1u);
-              const uint32_t sfb_t = sfa_t + 4u;
-              tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + (uint64_t)((s * kSfChunk) >> 4));
-              tc_cp_32x128b_warpx4(sfb_t, sfb_desc0 + (uint64_t)((s * kIdxSmemSFB) >> 4));
-              if (kN > 128)
-                tc_cp_32x128b_warpx4(sfb_t + 4u,
-                                     sfb_desc0 + (uint64_t)((s * kIdxSmemSFB + kSfChunk) >> 4));
-              const uint64_t adesc = a_desc0 + (uint64_t)((s * kIdxSmemA) >> 4);
-              const uint64_t bdesc = b_desc0 + (uint64_t)((s * kIdxSmemB) >> 4);
+    // This thread shares its SMSP with three epilogue warps and each of its
+    // instructions takes tens of cycles, while the tensor pipe waits for it;
+    // so it walks no tile list: it takes the key stages in ring order and
+    // reads from each stage's info word what to do around its MMAs.
+    if (lane == 0) {
+      int s = 0, b = 0, qs = 0, qe = -1;
+      uint32_t ph = 0, acc_ph = 0, q_ph = 0, x = 0;  // x: TMEM scale buffer, flips every stage
+      int kb = 0;
+      int sfb_tag0 = -1, sfb_tag1 = -1;  // query epoch * KB + kb whose scales each TMEM scale buffer holds
+      bool issued_any = false, ok = true;
+      const uint32_t idesc0 = idesc_mxf8f6f4(/*A E2M1*/ 5, /*B E4M3*/ 0, 128, kN);
+      uint32_t id[4];
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t id = idesc_with_sf_id(idesc0, kk, kk);
-                mma_mxf8f6f4(acc, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id,
-                             (kb | kk) != 0 ? 1u : 0u, sfa_t | ((uint32_t)kk << 30),
-                             sfb_t | ((uint32_t)kk << 30));
-              }
-              issued_any = true;
-              tc_commit(&empty[s]);
-            }
-            if (ok) {
-              tc_commit(&acc_full[b]);
-              ++ta;
-            }
+      for (int kk = 0; kk < 4; ++kk) id[kk] = idesc_with_sf_id(idesc0, kk, kk);
+      const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA)), q_desc0 = sdesc_sw128(smem_u32(sQ));
+      const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
+      uint64_t qdesc = q_desc0;
+      uint32_t sfb_base = 0;
+      for (;;) {
+        if (!mbar_wait_or_abort(&full[s], ph, kWaitLimitNs, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int info = sinfo[s];
+        if (info == kStEnd) break;
+        if (info == kStRelQ) {
+          // the current query slot is free once the MMAs issued so far complete
+          tc_commit(&q_empty[qs]);
+          if (++qs == NQ) {
+            qs = 0;
+            q_ph ^= 1u;
+          }
+          mbar_arrive(&empty[s]);  // the stage carried no data
+          if (++s == NS) {
+            s = 0;
+            ph ^= 1u;
+          }
+          continue;
+        }
+        if (info & kStNewQ) {
+          ++qe;
+          qdesc = q_desc0 + (uint64_t)(((uint32_t)qs * KB * kIdxQBlock) >> 4);
+          sfb_base = (uint32_t)qs * KB * kIdxSfbBlock;
+          if (!mbar_wait_or_abort(&q_full[qs], q_ph, 2 * kWaitLimitNs, abort_flag)) {
+            ok = false;
+            break;
           }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (info & kStFirst) {
+          kb = 0;
+          if (!mbar_wait_or_abort(&acc_empty[b], acc_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+            ok = false;
+            break;
+          }
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + kIdxAccStride * (uint32_t)b;
+        const uint32_t sfa_t = tmem + kIdxSfCol + 16u * x;
+        const uint32_t sfb_t = sfa_t + 4u;
+        tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + (uint64_t)(((uint32_t)s * kSfChunk) >> 4));
+        const int tag = qe * KB + kb;
+        if ((x ? sfb_tag1 : sfb_tag0) != tag) {  // else the buffer still holds these scales
+          const uint32_t sfb_off = sfb_base + (uint32_t)kb * kIdxSfbBlock;
+          tc_cp_32x128b_warpx4(sfb_t, sfb_desc0 + (uint64_t)(sfb_off >> 4));
+          if (kN > 128)
+            tc_cp_32x128b_warpx4(sfb_t + 4u, sfb_desc0 + (uint64_t)((sfb_off + kSfChunk) >> 4));
+          if (x)
+            sfb_tag1 = tag;
+          else
+            sfb_tag0 = tag;
+        }
+        const uint64_t adesc = a_desc0 + (uint64_t)(((uint32_t)s * kIdxSmemA) >> 4);
+        const uint64_t bdesc = qdesc + (uint64_t)(((uint32_t)kb * kIdxQBlock) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_mxf8f6f4(acc, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id[kk],
+                       (kb | kk) != 0 ? 1u : 0u, sfa_t | ((uint32_t)kk << 30),
+                       sfb_t | ((uint32_t)kk << 30));
+        issued_any = true;
+        tc_commit(&empty[s]);
+        if (info & kStLast) {
+          tc_commit(&acc_full[b]);
+          b ^= 1;
+          if (b == 0) acc_ph ^= 1u;
+        }
+        ++kb;
+        x ^= 1u;
+        if (++s == NS) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
-    }
-    if (lane == 0 && !ok) {
-      if (!*abort_flag) record_timeout(args.hdr, 120);
-      *abort_flag = 1;
-      if (issued_any) {  // wait for the MMAs in flight before TMEM is released
-        tc_commit(drain);
-        (void)mbar_wait(drain, 0);
+      if (!ok) {
+        if (!*abort_flag) record_timeout(args.hdr, 120);
+        *abort_flag = 1;
+        if (issued_any) {  // wait for the MMAs in flight before TMEM is released
+          tc_commit(drain);
+          (void)mbar_wait(drain, 0);
+        }
       }
     }
   } else {
@@ -307,14 +481,21 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     constexpr int kMine = (kTok + 2) / 3;
     int ta = 0;
     bool dead = false;
+    int unit_m = -1, g = 0, kt0 = 0;  // the current unit, looked up once per unit
     uint32_t fnext = act_flag(lane);
     for (long long k0 = 0; k0 < n_mine && !dead; k0 += 32) {
       const uint32_t mask = __ballot_sync(0xffffffffu, fnext != 0);
       fnext = act_flag(k0 + 32 + lane);
       const int nb = (int)(n_mine - k0 < 32 ? n_mine - k0 : 32);
       for (int bit = 0; bit < nb; ++bit) {
-        const int tile = tile_of(k0 + bit);
-        const int g = tile / args.n_tiles_k, kt = tile - g * args.n_tiles_k;
+        const long long k = k0 + bit;
+        const int m = (int)(k >> args.chunk_log2);
+        if (m != unit_m) {
+          unit_m = m;
+          (void)cta_unit(args, m, g, kt0);  // k < n_mine: the unit exists
+        }
+        const int kt = kt0 + (int)(k & ((1 << args.chunk_log2) - 1));
+        if (kt >= args.n_tiles_k) continue;  // past the last key tile: no entries
         const int j = kt * 128 + r;
         const bool active = (mask >> bit) & 1u;
         // key ranges of this warp's tokens (loaded before the waits)
@@ -419,10 +600,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   __syncthreads();
   if (warp == 0 && lane == 0 && *abort_flag) {
     // copies issued that nobody consumed land before the CTA's memory goes away
-    for (int s = 0; s < kIdxStages; ++s)
+    for (int s = 0; s < NS; ++s)
       if (issued_mask & (1u << s)) (void)mbar_wait(&full[s], (last_phase >> s) & 1);
     for (int b = 0; b < kIdxWSlots; ++b)
       if (w_issued & (1u << b)) (void)mbar_wait(&w_full[b], (w_phase >> b) & 1);
+    for (int b = 0; b < 2; ++b)
+      if (q_issued & (1u << b)) (void)mbar_wait(&q_full[b], (q_phase >> b) & 1);
   }
   if (warp == 1) {
     __syncwarp();
@@ -486,7 +669,7 @@ __global__ void q_sf_prep_kernel(const int32_t* __restrict__ q_sf, long long row
     const int kb = (int)(x - r * KB);
     const long long g = r / kN;
     const int rr = (int)(r - g * kN);
-    uint8_t* dst = out + ((size_t)g * KB + kb) * kIdxSmemSFB + (rr >> 7) * kSfChunk;
+    uint8_t* dst = out + ((size_t)g * KB + kb) * kIdxSfbBlock + (rr >> 7) * kSfChunk;
     const int r7 = rr & 127;
     *reinterpret_cast<int32_t*>(dst + (r7 & 31) * 16 + (r7 >> 5) * 4) = q_sf[x];
   }
@@ -495,7 +678,7 @@ __global__ void q_sf_prep_kernel(const int32_t* __restrict__ q_sf, long long row
 }  // namespace
 
 int mqa_tokens_per_tile(int Hh) { return idx_tokens(Hh); }
-size_t mqa_qsf_bytes_per_group(int D) { return (size_t)(D / 128) * kIdxSmemSFB; }
+size_t mqa_qsf_bytes_per_group(int D) { return (size_t)(D / 128) * kIdxSfbBlock; }
 
 cudaError_t launch_kv_prep(const uint8_t* kv, const uint8_t* kv_sf, int N, int Np, int D,
                            uint8_t* codes, uint8_t* chunks, cudaStream_t stream) {
@@ -539,7 +722,7 @@ cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, co
   if (!attr_set[slot]) {
     cudaError_t err = cudaFuncSetAttribute((const void*)fn,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)kIdxSmemBytes);
+                                           kIdxSmemMax);
     if (err != cudaSuccess) return err;
     attr_set[slot] = true;
   }
@@ -559,6 +742,17 @@ cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, co
   a.n_tiles_k = (N + 127) / 128;
   a.n_groups = (S + idx_tokens(Hh) - 1) / idx_tokens(Hh);
   a.act = act;
+  // key tiles per unit: 16, halved while the units would number fewer than
+  // four per CTA, and no more than the key tiles round up to
+  int lg = 4;
+  while (lg > 0 && ((long long)a.n_groups * ((a.n_tiles_k + (1 << lg) - 1) >> lg) < 4LL * grid ||
+                    (1 << (lg - 1)) >= a.n_tiles_k))
+    --lg;
+  a.chunk_log2 = lg;
+  a.n_chunks = (a.n_tiles_k + (1 << lg) - 1) >> lg;
+  a.n_units = a.n_groups * a.n_chunks;
+  const IdxSmem L = idx_smem(KB);
+  if (L.stages < 1 || L.total > kIdxSmemMax) return cudaErrorInvalidValue;
   {
     const long long tiles = (long long)a.n_tiles_k * a.n_groups;
     long long agrid = (tiles + 255) / 256;
@@ -571,7 +765,7 @@ cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, co
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kIdxThreads);
-  cfg.dynamicSmemBytes = kIdxSmemBytes;
+  cfg.dynamicSmemBytes = (size_t)L.total;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

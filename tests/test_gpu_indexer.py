@@ -83,6 +83,27 @@ def test_small_shapes_every_entry(S, Hh, D, N):
     _check(got, d, label=f"S{S} Hh{Hh} D{D} N{N}")
 
 
+@pytest.mark.parametrize("S,Hh,D,N,sms", [
+    (40, 16, 384, 1000, 3),   # 3 CTAs: several two-tile units and group changes each
+    (20, 64, 128, 700, 1),    # one CTA walks every tile: query slots and key ring wrap
+    (33, 32, 256, 129, 2),    # 2 K-blocks: seven key stages
+    (9, 128, 512, 400, 1),    # 4 K-blocks: a single query slot
+    (7, 64, 1024, 300, 2),    # 8 K-blocks: one query slot, one key stage
+])
+def test_few_ctas_many_tiles_each(S, Hh, D, N, sms):
+    """With the SM count capped, every CTA runs many tiles and query groups,
+    so the query slots, their scale buffers and the key ring are reused."""
+    import block_scaled_fp8_permute_b200 as moe
+    d = _inputs(S, Hh, D, N, seed=S * 7 + N)
+    moe.moe_set_num_sms(sms)
+    try:
+        got, st = _run(d)
+    finally:
+        moe.moe_set_num_sms(0)
+    assert st == 0
+    _check(got, d, label=f"S{S} Hh{Hh} D{D} N{N} sms{sms}")
+
+
 def test_without_cleaning_nothing_outside_the_ranges_is_written():
     d = _inputs(12, 64, 128, 500, seed=3)
     got, st = _run(d, clean=False, sentinel=12345.0)
