@@ -48,7 +48,8 @@ constexpr int kIdxQBlock = 192 * 128;  // one K-block of a query block (up to 19
 constexpr int kIdxSfbBlock = 2 * kSfChunk;  // the query scales of one K-block
 constexpr int kIdxTxA = 128 * 128 / 2; // bytes the TMA moves for the packed keys
 constexpr int kIdxEpiWarps = 12;  // three per 32-lane TMEM subpartition
-constexpr int kIdxThreads = 64 + 32 * kIdxEpiWarps;
+constexpr int kIdxMma2Warp = 2 + kIdxEpiWarps;  // the second MMA thread's warp (14)
+constexpr int kIdxThreads = 32 * (kIdxMma2Warp + 1);
 constexpr uint32_t kIdxTmemCols = 512;
 constexpr uint32_t kIdxAccStride = 256;  // accumulator buffer b at column 256 b
 constexpr uint32_t kIdxSfCol = 448;      // scale buffers: SFA at +16x (4 cols), SFB at +16x+4 (8)
@@ -56,12 +57,14 @@ constexpr int kIdxWSlot = 1024;          // the group's kN weights, up to 768 by
 constexpr int kIdxWSlots = 4;
 constexpr int kIdxSmemMax = 232448;      // shared memory per CTA
 constexpr int kIdxBarBytes = 512;
-// stage info words (producer -> MMA thread)
-constexpr int kStFirst = 1;   // the tile's first K-block: take the next accumulator buffer
-constexpr int kStLast = 2;    // the tile's last K-block: hand the accumulator to the epilogue
-constexpr int kStNewQ = 4;    // the tile starts a new query group: take the next query slot
-constexpr int kStEnd = 8;     // no more work (a stage without loads)
-constexpr int kStRelQ = 16;   // release the current query slot (a stage without loads)
+// Stage info word (producer -> MMA thread): bits 0-1 kind, then for a key
+// stage: bit 2 the tile's first K-block, bit 3 its last, bit 4 the parity of
+// the query slot's load, bit 5 the query slot, bits 8-15 kb, bits 16-31 the
+// query epoch (group change count) mod 2^16; for a release: bit 5 the slot.
+constexpr int kStKey = 0;     // a key stage of a tile
+constexpr int kStRelQ = 1;    // release a query slot (a stage without loads)
+constexpr int kStEnd = 2;     // no more work (a stage without loads)
+constexpr int kStFirst = 4, kStLast = 8, kStQPar = 16, kStQSlot = 32;
 static_assert(kIdxSmemA % 1024 == 0 && kIdxQBlock % 1024 == 0, "swizzled block alignment");
 
 // tokens per tile for Hh heads: kN = kTok * Hh query rows on the MMA's N side
@@ -187,12 +190,19 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint64_t* acc_empty = acc_full + 2;         // [2]
   uint64_t* w_full = acc_empty + 2;           // [kIdxWSlots] weight slot loaded
   uint64_t* w_empty = w_full + kIdxWSlots;    // [kIdxWSlots] weight slot read by every epilogue warp
-  uint64_t* drain = w_empty + kIdxWSlots;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = w_empty + kIdxWSlots;   // [2] one per MMA thread
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  // what the MMA thread does with key stage s (written by the producer before
+  // what the MMA thread does with stage s (written by the producer before
   // the stage's loads are issued; read after the stage's full barrier)
   int* sinfo = const_cast<int*>(abort_flag) + 1;  // [kIdxMaxStages]
+  // Two MMA threads (warp 1 and warp 14, on different SMSPs) take alternate
+  // active tiles, each with its own half of the key ring and its own
+  // accumulator buffer, so one thread's bookkeeping overlaps the other's
+  // MMAs.  With a single key stage (8 K-blocks) there is one ring and one
+  // MMA thread.
+  const int n_rings = NS >= 2 ? 2 : 1;
+  const int ring_a = n_rings == 2 ? (NS + 1) / 2 : NS;  // ring 0: stages [0, ring_a), ring 1: the rest
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&q_full[b], 1);
-      mbar_init(&q_empty[b], 1);
+      mbar_init(&q_empty[b], n_rings);
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kIdxEpiWarps);
     }
@@ -210,7 +220,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       mbar_init(&w_full[b], 1);
       mbar_init(&w_empty[b], kIdxEpiWarps);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -250,13 +261,59 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Ring positions advance by increments (no division on the per-tile
-    // path); the unit is looked up once per unit.
-    int s = 0, wb = 0, qs = 0;
-    uint32_t ph = 0, w_ph = 0, q_ph = 0;
+    // path); the unit is looked up once per unit.  Active tile number tp
+    // goes to key ring tp % n_rings.
+    struct Ring {
+      int s, lo, hi;
+      uint32_t ph;
+    };
+    Ring rg0{0, 0, ring_a, 0}, rg1{ring_a, ring_a, NS, 0};
+    int wb = 0, qs = 0, tp = 0;
+    uint32_t w_ph = 0, q_ph = 0;
     int qe = -1, cur_g = -1, cur_m = -1, g = 0, kt0 = 0;
     bool ok = true;
     const uint32_t tx = kIdxTxA + kSfChunk;
     const uint32_t qtx = (uint32_t)KB * (kN * 128 + kIdxSfbBlock);
+    // the next stage of ring R: wait for it to be free
+    auto take = [&](Ring& R, int site) -> bool {
+      if (!mbar_wait_or_abort(&empty[R.s], R.ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+        if (!*abort_flag) record_timeout(args.hdr, site);
+        *abort_flag = 1;
+        return false;
+      }
+      return true;
+    };
+    auto advance = [&](Ring& R) {
+      if (++R.s == R.hi) {
+        R.s = R.lo;
+        R.ph ^= 1u;
+      }
+    };
+    // a stage without loads: only its info word
+    auto send_info = [&](Ring& R, int code, int site) -> bool {
+      if (!take(R, site)) return false;
+      sinfo[R.s] = code;
+      mbar_arrive(&full[R.s]);
+      advance(R);
+      return true;
+    };
+    // the key stages of one tile
+    auto send_tile = [&](Ring& R, int kt, int qinfo) -> bool {
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!take(R, 110)) return false;
+        const int st = R.s;
+        sinfo[st] = kStKey | (kb == 0 ? kStFirst : 0) | (kb == KB - 1 ? kStLast : 0) | qinfo |
+                    (kb << 8);
+        mbar_arrive_expect_tx(&full[st], tx);
+        tma_load_3d(sA + (size_t)st * kIdxSmemA, &tmK, &full[st], 0, kt * 128, kb);
+        bulk_load(sSFA + st * kSfChunk, args.sfa + ((size_t)kb * args.n_tiles_k + kt) * kSfChunk,
+                  kSfChunk, &full[st]);
+        issued_mask |= 1u << st;
+        last_phase = (last_phase & ~(1u << st)) | (R.ph << st);
+        advance(R);
+      }
+      return true;
+    };
     uint32_t fnext = act_flag(lane);
     for (long long k0 = 0; k0 < n_mine && ok; k0 += 32) {
       uint32_t mask = __ballot_sync(0xffffffffu, fnext != 0);
@@ -271,68 +328,43 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             (void)cta_unit(args, m, g, kt0);  // an active tile: its unit exists
           }
           const int kt = kt0 + (int)(k & ((1 << args.chunk_log2) - 1));
-          const bool new_epoch = g != cur_g;
-          if (new_epoch && qe >= 0) {
-            // An info-only stage tells the MMA thread that the current query
-            // slot is read by no later MMA: it releases the slot once the MMAs
-            // issued so far complete.  (With one slot the wait below needs
-            // exactly that release.)
-            if (!mbar_wait_or_abort(&empty[s], ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
-              if (!*abort_flag) record_timeout(args.hdr, 114);
-              *abort_flag = 1;
-              ok = false;
-            } else {
-              sinfo[s] = kStRelQ;
-              mbar_arrive(&full[s]);
-              if (++s == NS) {
-                s = 0;
-                ph ^= 1u;
-              }
+          if (g != cur_g) {
+            if (qe >= 0) {
+              // Info-only stages tell both MMA threads that the current query
+              // slot is read by no later MMA: each releases it once its MMAs
+              // issued so far complete.  (With one slot the wait below needs
+              // exactly that release.)
+              const int code = kStRelQ | (qs ? kStQSlot : 0);
+              ok = send_info(rg0, code, 114) && (n_rings == 1 || send_info(rg1, code, 114));
               if (++qs == NQ) {
                 qs = 0;
                 q_ph ^= 1u;
               }
             }
-          }
-          if (new_epoch && ok) {
-            // a new query group: its query block and scales into the next slot
-            ++qe;
-            cur_g = g;
-            if (!mbar_wait_or_abort(&q_empty[qs], q_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
-              if (!*abort_flag) record_timeout(args.hdr, 112);
-              *abort_flag = 1;
-              ok = false;
-            } else {
-              mbar_arrive_expect_tx(&q_full[qs], qtx);
-              for (int kb = 0; kb < KB; ++kb)
-                tma_load_2d(sQ + (size_t)(qs * KB + kb) * kIdxQBlock, &tmQ, &q_full[qs], kb * 128,
-                            g * kN);
-              bulk_load(sSFB + (size_t)qs * KB * kIdxSfbBlock,
-                        args.sfb + (size_t)g * KB * kIdxSfbBlock, (uint32_t)KB * kIdxSfbBlock,
-                        &q_full[qs]);
-              q_issued |= 1u << qs;
-              q_phase = (q_phase & ~(1u << qs)) | (q_ph << qs);
+            if (ok) {
+              // a new query group: its query block and scales into the next slot
+              ++qe;
+              cur_g = g;
+              if (!mbar_wait_or_abort(&q_empty[qs], q_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+                if (!*abort_flag) record_timeout(args.hdr, 112);
+                *abort_flag = 1;
+                ok = false;
+              } else {
+                mbar_arrive_expect_tx(&q_full[qs], qtx);
+                for (int kb = 0; kb < KB; ++kb)
+                  tma_load_2d(sQ + (size_t)(qs * KB + kb) * kIdxQBlock, &tmQ, &q_full[qs],
+                              kb * 128, g * kN);
+                bulk_load(sSFB + (size_t)qs * KB * kIdxSfbBlock,
+                          args.sfb + (size_t)g * KB * kIdxSfbBlock, (uint32_t)KB * kIdxSfbBlock,
+                          &q_full[qs]);
+                q_issued |= 1u << qs;
+                q_phase = (q_phase & ~(1u << qs)) | (q_ph << qs);
+              }
             }
           }
-          for (int kb = 0; kb < KB && ok; ++kb) {
-            if (!mbar_wait_or_abort(&empty[s], ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
-              if (!*abort_flag) record_timeout(args.hdr, 110);
-              *abort_flag = 1;
-              ok = false;
-              break;
-            }
-            sinfo[s] = (kb == 0 ? kStFirst : 0) | (kb == KB - 1 ? kStLast : 0) |
-                       (kb == 0 && new_epoch ? kStNewQ : 0);
-            mbar_arrive_expect_tx(&full[s], tx);
-            tma_load_3d(sA + (size_t)s * kIdxSmemA, &tmK, &full[s], 0, kt * 128, kb);
-            bulk_load(sSFA + s * kSfChunk,
-                      args.sfa + ((size_t)kb * args.n_tiles_k + kt) * kSfChunk, kSfChunk, &full[s]);
-            issued_mask |= 1u << s;
-            last_phase = (last_phase & ~(1u << s)) | (ph << s);
-            if (++s == NS) {
-              s = 0;
-              ph ^= 1u;
-            }
+          if (ok) {
+            const int qinfo = (q_ph ? kStQPar : 0) | (qs ? kStQSlot : 0) | ((qe & 0xffff) << 16);
+            ok = (n_rings == 2 && (tp & 1)) ? send_tile(rg1, kt, qinfo) : send_tile(rg0, kt, qinfo);
           }
           if (ok) {
             // the group's weights into the next slot of the weight ring (rows
@@ -352,87 +384,72 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                 wb = 0;
                 w_ph ^= 1u;
               }
+              ++tp;
             }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
       }
     }
-    // one more stage, without loads, tells the MMA thread that the work ends
+    // one more stage per ring, without loads, tells the MMA threads that the work ends
     if (lane == 0 && ok) {
-      if (!mbar_wait_or_abort(&empty[s], ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
-        if (!*abort_flag) record_timeout(args.hdr, 113);
-        *abort_flag = 1;
-      } else {
-        sinfo[s] = kStEnd;
-        mbar_arrive(&full[s]);
-      }
+      if (send_info(rg0, kStEnd, 113) && n_rings == 2) (void)send_info(rg1, kStEnd, 113);
     }
-  } else if (warp == 1) {
+  } else if ((warp == 1 || (warp == kIdxMma2Warp && n_rings == 2)) && lane == 0) {
     // ----------------------------------------------------------------- MMA
-    // This thread shares its SMSP with three epilogue warps and each of its
-    // instructions takes tens of cycles, while the tensor pipe waits for it;
-    // so it walks no tile list: it takes the key stages in ring order and
+    // Each MMA thread shares its SMSP with three epilogue warps and each of
+    // its instructions takes tens of cycles while the tensor pipe waits for
+    // it; so it walks no tile list: it takes its ring's stages in order and
     // reads from each stage's info word what to do around its MMAs.
-    if (lane == 0) {
-      int s = 0, b = 0, qs = 0, qe = -1;
-      uint32_t ph = 0, acc_ph = 0, q_ph = 0, x = 0;  // x: TMEM scale buffer, flips every stage
-      int kb = 0;
-      int sfb_tag0 = -1, sfb_tag1 = -1;  // query epoch * KB + kb whose scales each TMEM scale buffer holds
-      bool issued_any = false, ok = true;
-      const uint32_t idesc0 = idesc_mxf8f6f4(/*A E2M1*/ 5, /*B E4M3*/ 0, 128, kN);
-      uint32_t id[4];
+    const int r = warp == 1 ? 0 : 1;  // ring, and (with two rings) accumulator buffer
+    const int lo = r == 0 ? 0 : ring_a, hi = r == 0 ? ring_a : NS;
+    int s = lo, b = r, cur_q = -1;
+    uint32_t ph = 0, acc_ph = 0, x = 0;  // x: which of this thread's two TMEM scale buffers
+    int sfb_tag0 = -1, sfb_tag1 = -1;  // (epoch << 8 | kb) + 1 whose query scales each scale buffer holds
+    bool issued_any = false, ok = true;
+    const uint32_t idesc0 = idesc_mxf8f6f4(/*A E2M1*/ 5, /*B E4M3*/ 0, 128, kN);
+    uint32_t id[4];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) id[kk] = idesc_with_sf_id(idesc0, kk, kk);
-      const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA)), q_desc0 = sdesc_sw128(smem_u32(sQ));
-      const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
-      uint64_t qdesc = q_desc0;
-      uint32_t sfb_base = 0;
-      for (;;) {
-        if (!mbar_wait_or_abort(&full[s], ph, kWaitLimitNs, abort_flag)) {
+    for (int kk = 0; kk < 4; ++kk) id[kk] = idesc_with_sf_id(idesc0, kk, kk);
+    const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA)), q_desc0 = sdesc_sw128(smem_u32(sQ));
+    const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
+    for (;;) {
+      if (!mbar_wait_or_abort(&full[s], ph, kWaitLimitNs, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const int info = sinfo[s];
+      const int kind = info & 3;
+      if (kind == kStEnd) break;
+      const int qs = (info & kStQSlot) ? 1 : 0;
+      if (kind == kStRelQ) {
+        // the query slot is free once this thread's MMAs issued so far complete
+        tc_commit(&q_empty[qs]);
+        mbar_arrive(&empty[s]);  // the stage carried no data
+      } else {
+        const int qtag = info >> 16;  // query epoch mod 2^16
+        if (qtag != cur_q) {
+          cur_q = qtag;
+          if (!mbar_wait_or_abort(&q_full[qs], (info & kStQPar) ? 1u : 0u, 2 * kWaitLimitNs,
+                                  abort_flag)) {
+            ok = false;
+            break;
+          }
+        }
+        if ((info & kStFirst) &&
+            !mbar_wait_or_abort(&acc_empty[b], acc_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
           ok = false;
           break;
         }
-        const int info = sinfo[s];
-        if (info == kStEnd) break;
-        if (info == kStRelQ) {
-          // the current query slot is free once the MMAs issued so far complete
-          tc_commit(&q_empty[qs]);
-          if (++qs == NQ) {
-            qs = 0;
-            q_ph ^= 1u;
-          }
-          mbar_arrive(&empty[s]);  // the stage carried no data
-          if (++s == NS) {
-            s = 0;
-            ph ^= 1u;
-          }
-          continue;
-        }
-        if (info & kStNewQ) {
-          ++qe;
-          qdesc = q_desc0 + (uint64_t)(((uint32_t)qs * KB * kIdxQBlock) >> 4);
-          sfb_base = (uint32_t)qs * KB * kIdxSfbBlock;
-          if (!mbar_wait_or_abort(&q_full[qs], q_ph, 2 * kWaitLimitNs, abort_flag)) {
-            ok = false;
-            break;
-          }
-        }
-        if (info & kStFirst) {
-          kb = 0;
-          if (!mbar_wait_or_abort(&acc_empty[b], acc_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
-            ok = false;
-            break;
-          }
-        }
         tc_fence_after();
+        const int kb = (info >> 8) & 0xff;
         const uint32_t acc = tmem + kIdxAccStride * (uint32_t)b;
-        const uint32_t sfa_t = tmem + kIdxSfCol + 16u * x;
+        const uint32_t sfa_t = tmem + kIdxSfCol + 16u * (2u * (uint32_t)r + x);
         const uint32_t sfb_t = sfa_t + 4u;
         tc_cp_32x128b_warpx4(sfa_t, sfa_desc0 + (uint64_t)(((uint32_t)s * kSfChunk) >> 4));
-        const int tag = qe * KB + kb;
-        if ((x ? sfb_tag1 : sfb_tag0) != tag) {  // else the buffer still holds these scales
-          const uint32_t sfb_off = sfb_base + (uint32_t)kb * kIdxSfbBlock;
+        const int tag = ((qtag << 8) | kb) + 1;
+        if ((x ? sfb_tag1 : sfb_tag0) != tag) {  // else the buffer still holds these query scales
+          const uint32_t sfb_off = (uint32_t)(qs * KB + kb) * kIdxSfbBlock;
           tc_cp_32x128b_warpx4(sfb_t, sfb_desc0 + (uint64_t)(sfb_off >> 4));
           if (kN > 128)
             tc_cp_32x128b_warpx4(sfb_t + 4u, sfb_desc0 + (uint64_t)((sfb_off + kSfChunk) >> 4));
@@ -442,7 +459,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             sfb_tag0 = tag;
         }
         const uint64_t adesc = a_desc0 + (uint64_t)(((uint32_t)s * kIdxSmemA) >> 4);
-        const uint64_t bdesc = qdesc + (uint64_t)(((uint32_t)kb * kIdxQBlock) >> 4);
+        const uint64_t bdesc = q_desc0 + (uint64_t)(((uint32_t)(qs * KB + kb) * kIdxQBlock) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_mxf8f6f4(acc, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id[kk],
@@ -452,26 +469,29 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         tc_commit(&empty[s]);
         if (info & kStLast) {
           tc_commit(&acc_full[b]);
-          b ^= 1;
-          if (b == 0) acc_ph ^= 1u;
+          if (n_rings == 1) {
+            b ^= 1;
+            if (b == 0) acc_ph ^= 1u;
+          } else {
+            acc_ph ^= 1u;
+          }
         }
-        ++kb;
         x ^= 1u;
-        if (++s == NS) {
-          s = 0;
-          ph ^= 1u;
-        }
       }
-      if (!ok) {
-        if (!*abort_flag) record_timeout(args.hdr, 120);
-        *abort_flag = 1;
-        if (issued_any) {  // wait for the MMAs in flight before TMEM is released
-          tc_commit(drain);
-          (void)mbar_wait(drain, 0);
-        }
+      if (++s == hi) {
+        s = lo;
+        ph ^= 1u;
       }
     }
-  } else {
+    if (!ok) {
+      if (!*abort_flag) record_timeout(args.hdr, 120 + r);
+      *abort_flag = 1;
+      if (issued_any) {  // wait for the MMAs in flight before TMEM is released
+        tc_commit(&drain[r]);
+        (void)mbar_wait(&drain[r], 0);
+      }
+    }
+  } else if (warp >= 2 && warp < kIdxMma2Warp) {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;          // 0..11
     const int q = warp & 3;           // TMEM lane subpartition this warp can read
