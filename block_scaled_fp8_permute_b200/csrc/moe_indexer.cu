@@ -22,15 +22,17 @@
 // CTA c takes units c, c + grid, ...  A CTA therefore meets the same query
 // group for up to C tiles in a row, and the group's query block (kN rows x D,
 // with its scales) is loaded once into a query slot and read by all of them;
-// only the 8 KB key tile streams per tile.  Without that, the query block was
-// most of the bytes a tile moved into shared memory, and the kernel was bound
-// by those loads.  One CTA per SM, persistent, 448 threads:
+// only the 8 KB key tile streams per tile (the 24 KB query block would
+// otherwise be most of a tile's bytes).  One CTA per SM, persistent, 480
+// threads:
 //   warp 0     TMA producer: query blocks into 1-2 query slots (one per group
 //              change), key tiles 128 x 128 (E2M1, unpacked by the TMA) with
 //              their scale chunk into a ring of up to 8 stages, and the
 //              group's head weights into a 4-deep weight ring
-//   warp 1     TMEM allocator and MMA issuer (tcgen05.mma kind::mxf8f6f4,
-//              A = keys E2M1, B = queries E4M3, M=128, N=kN, K=32)
+//   warps 1,14 TMEM allocator (warp 1) and two MMA-issuing threads
+//              (tcgen05.mma kind::mxf8f6f4, A = keys E2M1, B = queries E4M3,
+//              M=128, N=kN, K=32) taking alternate tiles, each with its own
+//              half of the key ring and its own accumulator buffer
 //   warps 2-13 epilogue: three warps per 32-lane TMEM subpartition, the
 //              group's tokens split between them
 // Tiles whose keys lie outside every token's [ks, ke) skip the loads and the

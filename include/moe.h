@@ -237,8 +237,8 @@ moe_status moe_forward_host_pipelined(const moe_shape* shape, int n_batches,
  *   - Shapes whose moe_workspace_bytes() exceeds 32 MiB are rejected with
  *     MOE_ERR_WORKSPACE before anything is launched (for example T = 256,
  *     H = 2048, I = 1024, E = 8, top-2 fits; the large workloads do not).
- *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *   - The first call on a device looks up the array's device address, with
+ *     that device current.
  *   - Nothing is allocated: no cudaMalloc, no cudaFree, no allocating
  *     library routine.  The header part of the array is cleared by every
  *     call; the rest keeps the last call's contents and is rewritten before
