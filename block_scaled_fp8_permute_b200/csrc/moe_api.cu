@@ -37,16 +37,13 @@ cudaError_t launch_gemm_prep(const int* masked_m, int G, int m_max, int mt_per_g
 
 cudaError_t launch_sf_chunks(const int32_t* a_sf, long long rows, int KG, uint8_t* sf_chunks,
                              cudaStream_t stream);
-cudaError_t launch_kv_prep(const uint8_t* kv, const uint8_t* kv_sf, int N, int Np, int D,
-                           uint8_t* codes, uint8_t* chunks, cudaStream_t stream);
 int mqa_tokens_per_tile(int Hh);
 size_t mqa_qsf_bytes_per_group(int D);
-cudaError_t launch_q_sf_prep(const int32_t* q_sf, long long rows, int D, int Hh, uint8_t* out,
-                             cudaStream_t stream);
-cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, const uint8_t* sfa,
-                              const uint8_t* sfb, const float* w, const int* ks, const int* ke,
-                              float* out, int* hdr, uint8_t* act, int S, int Hh, int N, int KB,
-                              int clean, int grid, bool pdl, cudaStream_t stream);
+cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, const uint8_t* kv,
+                              const uint8_t* kv_sf, uint8_t* codes, uint8_t* sfa, int Np,
+                              const int32_t* q_sf, uint8_t* sfb, const float* w, const int* ks,
+                              const int* ke, float* out, int* hdr, uint8_t* act, int S, int Hh,
+                              int N, int KB, int clean, int grid, bool pdl, cudaStream_t stream);
 
 namespace {
 
@@ -902,15 +899,13 @@ moe_status moe_fp8_fp4_mqa_logits(int S, int Hh, int D, int N, const uint8_t* q,
   if (!encode_wgt(&tmK, codes, 1, KB, L.Np, 128) ||
       !encode_act(&tmQ, q, S * Hh, D, mqa_tokens_per_tile(Hh) * Hh))
     return MOE_ERR_CUDA;
-  cudaError_t e = cudaMemsetAsync(hdr, 0, kHdrWords * 4, s);
-  if (e == cudaSuccess) e = launch_kv_prep(kv, kv_sf, N, L.Np, D, codes, kchunks, s);
-  if (e == cudaSuccess) e = launch_q_sf_prep(q_sf, (long long)S * Hh, D, Hh, qchunks, s);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  // two launches: the prep kernel (status words, key layout, query scale
+  // chunks, tile activity) and the logits kernel
   const long long tiles = (long long)(L.Np / 128) * L.n_groups;
   const int grid = (int)(tiles < sms ? tiles : sms);
-  return cuda_status(launch_mqa_logits(tmK, tmQ, kchunks, qchunks, weights, ks, ke, logits, hdr,
-                                       base + L.act, S, Hh, N, KB, clean ? 1 : 0, grid,
-                                       g_pdl.load() != 0, s));
+  return cuda_status(launch_mqa_logits(tmK, tmQ, kv, kv_sf, codes, kchunks, L.Np, q_sf, qchunks,
+                                       weights, ks, ke, logits, hdr, base + L.act, S, Hh, N, KB,
+                                       clean ? 1 : 0, grid, g_pdl.load() != 0, s));
 }
 
 moe_status moe_debug_requant(const float* a, int rows, int cols, uint8_t* codes, uint8_t* sbytes,

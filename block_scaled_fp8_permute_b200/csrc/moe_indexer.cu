@@ -173,6 +173,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   static_assert(kN % 16 == 0 && kN <= 192, "MMA N");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if ((smem_u32(smem_raw) & 1023u) != 0) {  // the swizzled layout needs it; no work done yet
+    pdl_wait();  // the status word is cleared by the previous kernel
     if (threadIdx.x == 0) set_status(args.hdr, MOE_ERR_CUDA);
     return;
   }
@@ -636,64 +637,76 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   }
 }
 
-// act[g * n_tiles_k + kt] = 1 when some token of query group g sees a key
-// of key tile kt.  One thread per tile.
-template <int kTok>
-__global__ void tile_activity_kernel(IdxArgs a, uint8_t* __restrict__ act) {
-  const long long total = (long long)a.n_groups * a.n_tiles_k;
-  for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total;
-       x += (long long)gridDim.x * blockDim.x) {
-    const int g = (int)(x / a.n_tiles_k), kt = (int)(x - (long long)g * a.n_tiles_k);
-    act[x] = tile_active<kTok>(a, kt, g) ? 1 : 0;
-  }
-}
-
 // Keys into the layout the key tiles stream, for any N: codes [KB][Np][64 B]
 // (Np = N rounded up to 128; padding rows zero) and UE8M0 chunks
 // [KB][Np/128][512 B] (byte (r%32)*16 + (r/32)*4 + j of a chunk = row r,
-// K-block j of the 128-element slice; padding rows zero).  One thread per
+// K-block j of the 128-element slice; padding rows zero).  Item x = one
 // (K-block, row).
-__global__ void kv_prep_kernel(const uint8_t* __restrict__ kv, const uint8_t* __restrict__ kv_sf,
-                               int N, int Np, int D, uint8_t* __restrict__ codes,
-                               uint8_t* __restrict__ chunks) {
-  const int KB = D / 128;
-  const long long total = (long long)KB * Np;
-  for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total;
-       x += (long long)gridDim.x * blockDim.x) {
-    const int n = (int)(x % Np), kb = (int)(x / Np);
-    uint4* d4 = reinterpret_cast<uint4*>(codes + ((size_t)kb * Np + n) * 64);
-    uint32_t sfw = 0;
-    if (n < N) {
-      const uint4* s4 = reinterpret_cast<const uint4*>(kv + (size_t)n * (D / 2) + (size_t)kb * 64);
+struct KvPrep {
+  const uint8_t* kv;
+  const uint8_t* kv_sf;
+  int N, Np, D;
+  uint8_t* codes;
+  uint8_t* chunks;
+};
+__device__ __forceinline__ void kv_prep_item(const KvPrep& p, long long x) {
+  const int n = (int)(x % p.Np), kb = (int)(x / p.Np);
+  uint4* d4 = reinterpret_cast<uint4*>(p.codes + ((size_t)kb * p.Np + n) * 64);
+  uint32_t sfw = 0;
+  if (n < p.N) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(p.kv + (size_t)n * (p.D / 2) + (size_t)kb * 64);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) d4[c] = s4[c];
-      sfw = *reinterpret_cast<const uint32_t*>(kv_sf + (size_t)n * (D / 32) + (size_t)kb * 4);
-    } else {
+    for (int c = 0; c < 4; ++c) d4[c] = s4[c];
+    sfw = *reinterpret_cast<const uint32_t*>(p.kv_sf + (size_t)n * (p.D / 32) + (size_t)kb * 4);
+  } else {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) d4[c] = make_uint4(0, 0, 0, 0);
-    }
-    const size_t chunk = (size_t)kb * (Np / 128) + (n >> 7);
-    *reinterpret_cast<uint32_t*>(chunks + chunk * kSfChunk + (n & 31) * 16 + ((n >> 5) & 3) * 4) = sfw;
+    for (int c = 0; c < 4; ++c) d4[c] = make_uint4(0, 0, 0, 0);
   }
+  const size_t chunk = (size_t)kb * (p.Np / 128) + (n >> 7);
+  *reinterpret_cast<uint32_t*>(p.chunks + chunk * kSfChunk + (n & 31) * 16 + ((n >> 5) & 3) * 4) = sfw;
 }
 
 // Query scales into per-group chunk pairs [group][KB][2][512 B]: query row r
 // (token * Hh + head) belongs to group r / kN, row rr = r % kN of it; chunk
 // rr / 128 of the pair, byte (rr%32)*16 + ((rr%128)/32)*4 + j.  Rows of the
 // pair past kN (or past the last token) stay whatever they were: their MMA
-// columns are never read.  One thread per (row, K-block).
-__global__ void q_sf_prep_kernel(const int32_t* __restrict__ q_sf, long long rows, int KB, int kN,
-                                 uint8_t* __restrict__ out) {
-  const long long total = rows * KB;
+// columns are never read.  Item x = one (row, K-block).
+struct QPrep {
+  const int32_t* q_sf;
+  int KB, kN;
+  uint8_t* out;
+};
+__device__ __forceinline__ void q_prep_item(const QPrep& p, long long x) {
+  const long long r = x / p.KB;
+  const int kb = (int)(x - r * p.KB);
+  const long long g = r / p.kN;
+  const int rr = (int)(r - g * p.kN);
+  uint8_t* dst = p.out + ((size_t)g * p.KB + kb) * kIdxSfbBlock + (rr >> 7) * kSfChunk;
+  const int r7 = rr & 127;
+  *reinterpret_cast<int32_t*>(dst + (r7 & 31) * 16 + (r7 >> 5) * 4) = p.q_sf[x];
+}
+
+// Everything the logits kernel reads that the call derives from its inputs,
+// in one launch: the status words cleared, the key layout, the query scale
+// chunks, and act[g * n_tiles_k + kt] = 1 when some token of query group g
+// sees a key of key tile kt.  The three jobs are independent; one grid-stride
+// loop walks their items back to back.
+template <int kTok>
+__global__ void mqa_prep_kernel(KvPrep kvp, long long n_kv, QPrep qp, long long n_q, IdxArgs a,
+                                uint8_t* __restrict__ act, long long n_act) {
+  if (blockIdx.x == 0 && threadIdx.x < kHdrWords) a.hdr[threadIdx.x] = 0;
+  const long long total = n_kv + n_q + n_act;
   for (long long x = blockIdx.x * (long long)blockDim.x + threadIdx.x; x < total;
        x += (long long)gridDim.x * blockDim.x) {
-    const long long r = x / KB;
-    const int kb = (int)(x - r * KB);
-    const long long g = r / kN;
-    const int rr = (int)(r - g * kN);
-    uint8_t* dst = out + ((size_t)g * KB + kb) * kIdxSfbBlock + (rr >> 7) * kSfChunk;
-    const int r7 = rr & 127;
-    *reinterpret_cast<int32_t*>(dst + (r7 & 31) * 16 + (r7 >> 5) * 4) = q_sf[x];
+    if (x < n_kv) {
+      kv_prep_item(kvp, x);
+    } else if (x < n_kv + n_q) {
+      q_prep_item(qp, x - n_kv);
+    } else {
+      const long long y = x - n_kv - n_q;
+      const int g = (int)(y / a.n_tiles_k), kt = (int)(y - (long long)g * a.n_tiles_k);
+      act[y] = tile_active<kTok>(a, kt, g) ? 1 : 0;
+    }
   }
 }
 
@@ -702,42 +715,21 @@ __global__ void q_sf_prep_kernel(const int32_t* __restrict__ q_sf, long long row
 int mqa_tokens_per_tile(int Hh) { return idx_tokens(Hh); }
 size_t mqa_qsf_bytes_per_group(int D) { return (size_t)(D / 128) * kIdxSfbBlock; }
 
-cudaError_t launch_kv_prep(const uint8_t* kv, const uint8_t* kv_sf, int N, int Np, int D,
-                           uint8_t* codes, uint8_t* chunks, cudaStream_t stream) {
-  const long long total = (long long)(D / 128) * Np;
-  if (total == 0) return cudaSuccess;
-  long long grid = (total + 255) / 256;
-  if (grid > 148LL * 32) grid = 148LL * 32;
-  kv_prep_kernel<<<(unsigned)grid, 256, 0, stream>>>(kv, kv_sf, N, Np, D, codes, chunks);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_q_sf_prep(const int32_t* q_sf, long long rows, int D, int Hh, uint8_t* out,
-                             cudaStream_t stream) {
-  const int KB = D / 128;
-  const long long total = rows * KB;
-  if (total == 0) return cudaSuccess;
-  long long grid = (total + 255) / 256;
-  if (grid > 148LL * 16) grid = 148LL * 16;
-  q_sf_prep_kernel<<<(unsigned)grid, 256, 0, stream>>>(q_sf, rows, KB,
-                                                       idx_tokens(Hh) * Hh, out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, const uint8_t* sfa,
-                              const uint8_t* sfb, const float* w, const int* ks, const int* ke,
-                              float* out, int* hdr, uint8_t* act, int S, int Hh, int N, int KB,
-                              int clean, int grid, bool pdl, cudaStream_t stream) {
+cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, const uint8_t* kv,
+                              const uint8_t* kv_sf, uint8_t* codes, uint8_t* sfa, int Np,
+                              const int32_t* q_sf, uint8_t* sfb, const float* w, const int* ks,
+                              const int* ke, float* out, int* hdr, uint8_t* act, int S, int Hh,
+                              int N, int KB, int clean, int grid, bool pdl, cudaStream_t stream) {
   typedef void (*Fn)(CUtensorMap, CUtensorMap, IdxArgs);
-  typedef void (*ActFn)(IdxArgs, uint8_t*);
+  typedef void (*ActFn)(KvPrep, long long, QPrep, long long, IdxArgs, uint8_t*, long long);
   Fn fn;
   ActFn afn;
   int slot;
   switch (Hh) {
-    case 16: fn = mqa_logits_kernel<16>; afn = tile_activity_kernel<idx_tokens(16)>; slot = 0; break;
-    case 32: fn = mqa_logits_kernel<32>; afn = tile_activity_kernel<idx_tokens(32)>; slot = 1; break;
-    case 64: fn = mqa_logits_kernel<64>; afn = tile_activity_kernel<idx_tokens(64)>; slot = 2; break;
-    case 128: fn = mqa_logits_kernel<128>; afn = tile_activity_kernel<idx_tokens(128)>; slot = 3; break;
+    case 16: fn = mqa_logits_kernel<16>; afn = mqa_prep_kernel<idx_tokens(16)>; slot = 0; break;
+    case 32: fn = mqa_logits_kernel<32>; afn = mqa_prep_kernel<idx_tokens(32)>; slot = 1; break;
+    case 64: fn = mqa_logits_kernel<64>; afn = mqa_prep_kernel<idx_tokens(64)>; slot = 2; break;
+    case 128: fn = mqa_logits_kernel<128>; afn = mqa_prep_kernel<idx_tokens(128)>; slot = 3; break;
     default: return cudaErrorInvalidValue;
   }
   static bool attr_set[4] = {};
@@ -776,11 +768,14 @@ cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, co
   const IdxSmem L = idx_smem(KB);
   if (L.stages < 1 || L.total > kIdxSmemMax) return cudaErrorInvalidValue;
   {
-    const long long tiles = (long long)a.n_tiles_k * a.n_groups;
-    long long agrid = (tiles + 255) / 256;
-    if (agrid > 148LL * 8) agrid = 148LL * 8;
-    if (agrid < 1) agrid = 1;
-    afn<<<(unsigned)agrid, 256, 0, stream>>>(a, act);
+    const KvPrep kvp{kv, kv_sf, N, Np, KB * 128, codes, sfa};
+    const QPrep qp{q_sf, KB, idx_tokens(Hh) * Hh, sfb};
+    const long long n_kv = (long long)KB * Np, n_q = (long long)S * Hh * KB;
+    const long long n_act = (long long)a.n_tiles_k * a.n_groups;
+    long long pgrid = (n_kv + n_q + n_act + 255) / 256;
+    if (pgrid > 148LL * 16) pgrid = 148LL * 16;
+    if (pgrid < 1) pgrid = 1;
+    afn<<<(unsigned)pgrid, 256, 0, stream>>>(kvp, n_kv, qp, n_q, a, act, n_act);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
   }
