@@ -43,7 +43,9 @@ cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, co
                               const uint8_t* kv_sf, uint8_t* codes, uint8_t* sfa, int Np,
                               const int32_t* q_sf, uint8_t* sfb, const float* w, const int* ks,
                               const int* ke, float* out, int* hdr, uint8_t* act, int S, int Hh,
-                              int N, int KB, int clean, int grid, bool pdl, cudaStream_t stream);
+                              int N, int KB, int clean, int grid, bool pdl,
+                              unsigned long long wait_limit_ns, int fault_skip_tile,
+                              cudaStream_t stream);
 
 namespace {
 
@@ -905,7 +907,8 @@ moe_status moe_fp8_fp4_mqa_logits(int S, int Hh, int D, int N, const uint8_t* q,
   const int grid = (int)(tiles < sms ? tiles : sms);
   return cuda_status(launch_mqa_logits(tmK, tmQ, kv, kv_sf, codes, kchunks, L.Np, q_sf, qchunks,
                                        weights, ks, ke, logits, hdr, base + L.act, S, Hh, N, KB,
-                                       clean ? 1 : 0, grid, g_pdl.load() != 0, s));
+                                       clean ? 1 : 0, grid, g_pdl.load() != 0,
+                                       g_fault_wait_ns.load(), g_fault_skip_it.load(), s));
 }
 
 moe_status moe_debug_requant(const float* a, int rows, int cols, uint8_t* codes, uint8_t* sbytes,

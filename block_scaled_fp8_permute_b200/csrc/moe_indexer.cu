@@ -113,6 +113,8 @@ struct IdxArgs {
   int chunk_log2;        // C = 2^chunk_log2 key tiles per unit (1..16)
   int n_chunks;          // ceil(n_tiles_k / C)
   int n_units;           // n_groups * n_chunks (< 2^28 for the supported shapes)
+  unsigned long long wait_limit_ns;  // 0: the default limits (a test hook shortens them)
+  int fault_skip_tile;   // test hook: 1 + the active tile whose key stage is never filled (0 = off)
 };
 
 // Does any token of query group g see a key of key tile kt?  (Decided the
@@ -179,6 +181,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   }
   const int KB = args.KB;
   const IdxSmem L = idx_smem(KB);
+  const unsigned long long lim = args.wait_limit_ns ? args.wait_limit_ns : kWaitLimitNs;
   const int NS = L.stages, NQ = L.qslots;
   uint8_t* sA = smem_raw + L.a_off;      // [NS][128 x 128]
   uint8_t* sQ = smem_raw + L.q_off;      // [NQ][KB][kN x 128]
@@ -279,7 +282,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const uint32_t qtx = (uint32_t)KB * (kN * 128 + kIdxSfbBlock);
     // the next stage of ring R: wait for it to be free
     auto take = [&](Ring& R, int site) -> bool {
-      if (!mbar_wait_or_abort(&empty[R.s], R.ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+      if (!mbar_wait_or_abort(&empty[R.s], R.ph ^ 1u, 2 * lim, abort_flag)) {
         if (!*abort_flag) record_timeout(args.hdr, site);
         *abort_flag = 1;
         return false;
@@ -303,6 +306,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // the key stages of one tile
     auto send_tile = [&](Ring& R, int kt, int qinfo) -> bool {
       for (int kb = 0; kb < KB; ++kb) {
+        if (kb == 0 && tp + 1 == args.fault_skip_tile) {  // test hook: this stage never fills
+          advance(R);
+          continue;
+        }
         if (!take(R, 110)) return false;
         const int st = R.s;
         sinfo[st] = kStKey | (kb == 0 ? kStFirst : 0) | (kb == KB - 1 ? kStLast : 0) | qinfo |
@@ -348,7 +355,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
               // a new query group: its query block and scales into the next slot
               ++qe;
               cur_g = g;
-              if (!mbar_wait_or_abort(&q_empty[qs], q_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+              if (!mbar_wait_or_abort(&q_empty[qs], q_ph ^ 1u, 2 * lim, abort_flag)) {
                 if (!*abort_flag) record_timeout(args.hdr, 112);
                 *abort_flag = 1;
                 ok = false;
@@ -372,7 +379,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           if (ok) {
             // the group's weights into the next slot of the weight ring (rows
             // of tokens past S are not read: the slot keeps stale values there)
-            if (!mbar_wait_or_abort(&w_empty[wb], w_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+            if (!mbar_wait_or_abort(&w_empty[wb], w_ph ^ 1u, 2 * lim, abort_flag)) {
               if (!*abort_flag) record_timeout(args.hdr, 111);
               *abort_flag = 1;
               ok = false;
@@ -417,7 +424,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const uint64_t a_desc0 = sdesc_sw128(smem_u32(sA)), q_desc0 = sdesc_sw128(smem_u32(sQ));
     const uint64_t sfa_desc0 = sdesc_sf(smem_u32(sSFA)), sfb_desc0 = sdesc_sf(smem_u32(sSFB));
     for (;;) {
-      if (!mbar_wait_or_abort(&full[s], ph, kWaitLimitNs, abort_flag)) {
+      if (!mbar_wait_or_abort(&full[s], ph, lim, abort_flag)) {
         ok = false;
         break;
       }
@@ -433,14 +440,14 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         const int qtag = info >> 16;  // query epoch mod 2^16
         if (qtag != cur_q) {
           cur_q = qtag;
-          if (!mbar_wait_or_abort(&q_full[qs], (info & kStQPar) ? 1u : 0u, 2 * kWaitLimitNs,
+          if (!mbar_wait_or_abort(&q_full[qs], (info & kStQPar) ? 1u : 0u, 2 * lim,
                                   abort_flag)) {
             ok = false;
             break;
           }
         }
         if ((info & kStFirst) &&
-            !mbar_wait_or_abort(&acc_empty[b], acc_ph ^ 1u, 2 * kWaitLimitNs, abort_flag)) {
+            !mbar_wait_or_abort(&acc_empty[b], acc_ph ^ 1u, 2 * lim, abort_flag)) {
           ok = false;
           break;
         }
@@ -537,8 +544,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
           const uint32_t par = (ta >> 1) & 1, wpar = (uint32_t)(ta / kIdxWSlots) & 1u;
           const bool ready =
               __all_sync(0xffffffffu,
-                         mbar_wait_or_abort(&acc_full[b], par, 2 * kWaitLimitNs, abort_flag) &&
-                             mbar_wait_or_abort(&w_full[wb], wpar, 2 * kWaitLimitNs, abort_flag));
+                         mbar_wait_or_abort(&acc_full[b], par, 2 * lim, abort_flag) &&
+                             mbar_wait_or_abort(&w_full[wb], wpar, 2 * lim, abort_flag));
           if (!ready) {
             if (lane == 0) {
               if (!*abort_flag) record_timeout(args.hdr, 130);
@@ -719,7 +726,9 @@ cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, co
                               const uint8_t* kv_sf, uint8_t* codes, uint8_t* sfa, int Np,
                               const int32_t* q_sf, uint8_t* sfb, const float* w, const int* ks,
                               const int* ke, float* out, int* hdr, uint8_t* act, int S, int Hh,
-                              int N, int KB, int clean, int grid, bool pdl, cudaStream_t stream) {
+                              int N, int KB, int clean, int grid, bool pdl,
+                              unsigned long long wait_limit_ns, int fault_skip_tile,
+                              cudaStream_t stream) {
   typedef void (*Fn)(CUtensorMap, CUtensorMap, IdxArgs);
   typedef void (*ActFn)(KvPrep, long long, QPrep, long long, IdxArgs, uint8_t*, long long);
   Fn fn;
@@ -765,6 +774,8 @@ cudaError_t launch_mqa_logits(const CUtensorMap& tmK, const CUtensorMap& tmQ, co
   a.chunk_log2 = lg;
   a.n_chunks = (a.n_tiles_k + (1 << lg) - 1) >> lg;
   a.n_units = a.n_groups * a.n_chunks;
+  a.wait_limit_ns = wait_limit_ns;
+  a.fault_skip_tile = fault_skip_tile;
   const IdxSmem L = idx_smem(KB);
   if (L.stages < 1 || L.total > kIdxSmemMax) return cudaErrorInvalidValue;
   {

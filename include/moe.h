@@ -264,7 +264,11 @@ moe_status moe_get_device_status(const void* workspace, moe_stream_t stream);
  * 20 + j the MMA issuer, 30 + j the epilogue warps of the one-SM grouped
  * GEMM, with j = 1 for linear1, 2 for linear2, 3 for the standalone GEMM;
  * 40 + j, 50 + j, 60 + j the same roles in the SM-pair kernel; 70 + j,
- * 80 + j, 90 + j in the swapped-role kernel.  -1 if the stream failed.
+ * 80 + j, 90 + j in the swapped-role kernel; in the FP4 indexer 110-114 the
+ * producer (key stage, weight slot, query slot, end, query-slot release),
+ * 120 / 121 the first / second MMA thread, 130 the epilogue warps (the same
+ * workspace word, read after moe_fp8_fp4_mqa_logits).  -1 if the stream
+ * failed.
  * Every wait on another role of the kernel is bounded (2 s for a stage's
  * data, 4 s for the waits that can only end after such a stage); when one
  * expires the kernel records MOE_ERR_TIMEOUT and this site, the other roles
@@ -278,7 +282,10 @@ int moe_get_timeout_site(const void* workspace, moe_stream_t stream);
  * kernel (one-SM tiles, normal m-tiles) skips the loads of its pipeline
  * iteration `skip_iteration` (-1: off), and the waits of that kernel use
  * `wait_limit_ns` for a stage's data and twice that otherwise (0: the
- * defaults above).  Process-wide; both off by default. */
+ * defaults above).  In every following moe_fp8_fp4_mqa_logits the producer
+ * of each CTA leaves the first key stage of its active tile number
+ * `skip_iteration` unfilled, with the same wait limits.  Process-wide; both
+ * off by default. */
 void moe_debug_set_fault(int skip_iteration, unsigned long long wait_limit_ns);
 
 /* Copies the plan out of `workspace` for bit-exact checking (synchronises

@@ -61,3 +61,51 @@ def test_expired_wait_is_reported_and_the_next_forward_is_correct(skip_iteration
     y_ref, _, _ = oracle.moe_forward(**d)
     assert_parity(y, y_ref, "after timeout")
     assert np.isfinite((y.astype(np.uint32) << 16).view(np.float32)).all()
+
+
+SITE_MMA_INDEXER = {0: 120, 1: 121}   # the MMA thread of ring 0 / ring 1
+
+
+@pytest.mark.parametrize("skip_tile", [0, 1])
+def test_indexer_expired_wait_is_reported_and_the_next_call_is_correct(skip_tile):
+    """The FP4 indexer's producer leaves the key stage of one active tile
+    unfilled (tile 0 goes to the first MMA thread's ring, tile 1 to the
+    second's); that thread's bounded wait expires, the call reports
+    MOE_ERR_TIMEOUT with its site, and the next call on the same workspace
+    matches the oracle."""
+    import time
+
+    import torch
+
+    import block_scaled_fp8_permute_b200 as moe
+    from tests.test_gpu_indexer import _check, _inputs
+
+    d = _inputs(20, 64, 128, 700, seed=5)
+    S, Hh, D = d["q"].shape
+    N = d["kv"].shape[0]
+    dev = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in d.items()}
+    out = torch.full((S, N), float("nan"), dtype=torch.float32, device="cuda")
+    ws = moe.alloc_mqa_workspace(S, Hh, D, N, "cuda")
+
+    def call():
+        moe.moe_fp8_fp4_mqa_logits(dev["q"], dev["q_sf"], dev["kv"], dev["kv_sf"], dev["weights"],
+                                   dev["ks"], dev["ke"], out, ws)
+    moe.moe_set_num_sms(2)   # two CTAs, about twenty tiles each
+    try:
+        moe.moe_debug_set_fault(skip_tile, 1_000_000)   # 1 ms
+        t0 = time.perf_counter()
+        call()
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+        moe.moe_debug_set_fault(-1, 0)
+        assert moe.moe_get_device_status(ws) == MOE_ERR_TIMEOUT
+        assert moe.moe_get_timeout_site(ws) == SITE_MMA_INDEXER[skip_tile]
+        assert elapsed < 1.0
+        call()
+        torch.cuda.synchronize()
+        assert moe.moe_get_device_status(ws) == 0
+        assert moe.moe_get_timeout_site(ws) == 0
+        _check(out.cpu().numpy(), d, label=f"after timeout, skip {skip_tile}")
+    finally:
+        moe.moe_debug_set_fault(-1, 0)
+        moe.moe_set_num_sms(0)
