@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  pdl_wait();  // the transformed keys and the query scale chunks come from the previous kernels
+  pdl_wait();  // the key layout, query scale chunks and tile activity come from the prep kernel
   uint32_t issued_mask = 0, last_phase = 0;  // key stages loaded (producer lane), for the failure path
   uint32_t w_issued = 0, w_phase = 0;        // weight slots loaded
   uint32_t q_issued = 0, q_phase = 0;        // query slots loaded
