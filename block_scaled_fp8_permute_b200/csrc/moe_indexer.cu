@@ -578,6 +578,13 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                 load_head_cols<kC>(trow + kIdxAccStride * (uint32_t)b +
                                        (uint32_t)((h + 3 * m) * kHh + c0), v[m]);
             tc_wait_ld();
+            if (c0 + kC >= kHh) {
+              // the last chunk is in registers: the accumulator buffer is free
+              // for the next tile's MMAs while the sums below run
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&acc_empty[b]);
+            }
 #pragma unroll
             for (int m = 0; m < kMine; ++m) {
               const int t = h + 3 * m;
@@ -595,13 +602,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             }
           }
         }
-        if (use) {  // accumulator and weights are in registers: release both
-          tc_fence_before();
+        if (use) {  // the weights are read: release their slot
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&acc_empty[b]);
-            mbar_arrive(&w_empty[wb]);
-          }
+          if (lane == 0) mbar_arrive(&w_empty[wb]);
         }
 #pragma unroll
         for (int m = 0; m < kMine; ++m) {
