@@ -89,6 +89,8 @@ def test_small_shapes_every_entry(S, Hh, D, N):
     (33, 32, 256, 129, 2),    # 2 K-blocks: seven key stages
     (9, 128, 512, 400, 1),    # 4 K-blocks: a single query slot
     (7, 64, 1024, 300, 2),    # 8 K-blocks: one query slot, one key stage
+    (6, 128, 128, 2000, 1),   # 128 heads: one token per tile, two TMEM load chunks per warp
+    (14, 32, 128, 900, 2),    # 32 heads: six tokens per tile, two per epilogue warp
 ])
 def test_few_ctas_many_tiles_each(S, Hh, D, N, sms):
     """With the SM count capped, every CTA runs many tiles and query groups,
